@@ -1,0 +1,558 @@
+"""Benchmark: prefill attention TFLOP/s and paged-decode KV GB/s on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill half: ragged THD causal prefill, 64 sequences with lengths
+    U[128, 8192], Hq/Hkv 32/8, D 128, per-batch padded LSE seeded -inf
+    (device work list, padded-LSE fill, tcgen05 prefill kernel);
+  * decode half: paged-KV decode, batch 128, KV lengths U[1024, 32768], page
+    64 with a random page permutation, Hq/Hkv 64/8, D 128, split-KV + LSE merge.
+`value` is the prefill half's TFLOP/s (the headline); the decode half is
+reported beside it under "decode".  Every input is larger than L2 (126 MB), so
+no flush is needed between timed steps.  Also measured per run: the dense
+causal prefill (B 8, S 4096) and the absorbed-MLA decode (B 64, 576/512).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own independently seeded batch of
+the same shape (weak scaling, no data-path collective); rank 0 prints the
+JSON line with the device time maxed over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill attention TFLOPS and paged-decode KV GB/s, % of B200 roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------------------- #
+# workload sizes (algorithmic units)
+# --------------------------------------------------------------------------- #
+def prefill_flops(lq, lkv, Hq, D, causal=True):
+    """4 * D flops per visible (query, key) pair per query head (QK^T and PV)."""
+    tot = 0
+    for a, b in zip(lq, lkv):
+        a, b = int(a), int(b)
+        if causal:
+            # rows i see min(b, i + b - a + 1) keys (bottom-right)
+            i = np.arange(a, dtype=np.int64)
+            tot += int(np.clip(i + b - a + 1, 0, b).sum())
+        else:
+            tot += a * b
+    return 4.0 * D * Hq * tot
+
+
+def decode_kv_bytes(kv_lens, Hkv, Dqk, Dv, alias):
+    per_tok = Hkv * (Dqk if alias else Dqk + Dv) * 2
+    return float(np.sum(np.asarray(kv_lens, dtype=np.int64)) * per_tok)
+
+
+# --------------------------------------------------------------------------- #
+# clocks sampler
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- #
+# our implementation
+# --------------------------------------------------------------------------- #
+class Part:
+    """One half of the hot path: inputs resident on the device plus a step()."""
+
+    def __init__(self, name, unit, units_per_step, launches_per_step, step, e2e=None, info=None):
+        self.name, self.unit, self.units = name, unit, units_per_step
+        self.launches = launches_per_step
+        self.step = step
+        self.e2e = e2e
+        self.info = info or {}
+
+
+def make_ragged_prefill(torch, rsd, synth, dev, seed_offset):
+    w = synth.WORKLOADS["ragged_prefill"]
+    L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
+    q, k, v, cu = synth.make_ragged(w, dev, lengths=L)
+    T = q.shape[0]
+    smax = int(L.max())
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, smax, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(rsd.attn_fwd_ragged_workspace_size(w.B, smax, T, w.Hq, w.Hkv), dtype=torch.uint8,
+                     device=dev)
+    cud = torch.as_tensor(cu, device=dev)
+
+    def step(qq=q, kk=k, vv=v, oo=o, ll=lse, cc=cud):
+        rsd.attn_fwd_ragged(qq, kk, vv, oo, ll, cc, cc, max_seqlen_q=smax, max_seqlen_kv=smax,
+                            scale=w.scale, causal=True, workspace=ws)
+
+    def e2e_setup():
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hcu = torch.as_tensor(cu).pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dcu = torch.empty_like(cud)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dcu.copy_(hcu, non_blocking=True)
+            step(dq, dk, dv, o, lse, dcu)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hcu))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        return e2e_step, h2d, d2h
+
+    flops = prefill_flops(L, L, w.Hq, w.Dqk)
+    info = {"workload": w.notes, "B": w.B, "total_tokens": int(T), "max_seqlen": smax,
+            "Hq": w.Hq, "Hkv": w.Hkv, "D": w.Dqk, "flop_per_step": flops,
+            "flop_per_unit": "4*D per visible (query, key) pair per query head"}
+    data = dict(q=q, k=k, v=v, cu=cu, L=L, w=w)
+    return Part("ragged_prefill", "TFLOP/s", flops / 1e12, 3, step, e2e_setup, info), data
+
+
+def make_dense_prefill(torch, rsd, synth, dev, seed_offset):
+    w = synth.WORKLOADS["dense_prefill"]
+    g = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+    q, k, v = synth.make_dense(g, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+
+    def step():
+        rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True)
+    flops = prefill_flops([w.S] * w.B, [w.S] * w.B, w.Hq, w.Dqk)
+    info = {"workload": w.notes, "flop_per_step": flops}
+    return Part("dense_prefill", "TFLOP/s", flops / 1e12, 1, step, None, info), None
+
+
+def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms):
+    w = synth.WORKLOADS[name]
+    L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
+    q, kp, vp, table, kl = synth.make_paged(w, dev, kv_lens=L)
+    Dv = w.Dv
+    o = torch.empty((w.B, w.Hq, Dv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    maxL = int(L.max())
+    S = rsd.attn_paged_suggest_splits(w.B, w.Hq, w.Hkv, w.Dqk, Dv, maxL, w.page_size, num_sms)
+    ws_n = rsd.attn_fwd_paged_workspace_size(w.B, w.Hq, Dv, S)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=dev)
+    pt = torch.as_tensor(table, device=dev)
+    kld = torch.as_tensor(kl, device=dev)
+
+    def step(qq=q, kk=kp, vv=vp, ptt=pt, kll=kld):
+        rsd.attn_fwd_paged(qq, kk, vv, o, lse, ptt, kll, page_size=w.page_size, max_kv_len=maxL,
+                           scale=w.scale, num_splits=S, workspace=ws)
+
+    def e2e_setup():
+        hq = q.cpu().pin_memory()
+        hk = kp.cpu().pin_memory()
+        hv = hk if w.v_aliases_k else vp.cpu().pin_memory()
+        hpt = pt.cpu().pin_memory()
+        hkl = kld.cpu().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq, dk = torch.empty_like(q), torch.empty_like(kp)
+        dv = dk if w.v_aliases_k else torch.empty_like(vp)
+        dpt, dkl = torch.empty_like(pt), torch.empty_like(kld)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            if not w.v_aliases_k:
+                dv.copy_(hv, non_blocking=True)
+            dpt.copy_(hpt, non_blocking=True)
+            dkl.copy_(hkl, non_blocking=True)
+            step(dq, dk, dv, dpt, dkl)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+        srcs = [hq, hk, hpt, hkl] + ([] if w.v_aliases_k else [hv])
+        h2d = sum(t.numel() * t.element_size() for t in srcs)
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+        return e2e_step, h2d, d2h
+
+    nbytes = decode_kv_bytes(L, w.Hkv, w.Dqk, Dv, w.v_aliases_k)
+    flops = float(np.sum(L)) * w.Hq * 2.0 * (w.Dqk + Dv)
+    info = {"workload": w.notes, "num_splits": S, "kv_bytes_per_step": nbytes,
+            "flop_per_step": flops, "total_pages": int(kp.shape[0]),
+            "bytes_per_unit": f"{w.Hkv * (w.Dqk if w.v_aliases_k else w.Dqk + Dv) * 2} B of K/V per cached token"}
+    data = dict(q=q, kp=kp, vp=vp, table=table, L=L, w=w, S=S)
+    launches = 2 if S > 1 else 1
+    return Part(name, "GB/s", nbytes / 1e9, launches, step, e2e_setup, info), data
+
+
+def time_part(torch, part, steps, warmup, dist, world):
+    """Device time of `steps` back-to-back steps (barrier + sync on both sides),
+    max over ranks; also per-step event durations on the launching stream."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        part.step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        part.step()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    total_ms = ev[0].elapsed_time(ev[-1])
+    per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    return total_ms, per
+
+
+def time_e2e(torch, part, steps, dist):
+    e2e_step, h2d, d2h = part.e2e()
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        e2e_step()
+        stream.synchronize()  # the step's result is read back on the host
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, h2d, d2h
+
+
+def oracle_prefill_sample(data, seconds):
+    """The fp64 oracle on a random sample of rows of the prefill batch.
+    Returns (TFLOP/s, threads, description)."""
+    import oracle
+    import synth
+    w, L, cu = data["w"], data["L"], data["cu"]
+    orc = oracle.default()
+    qb, kb, vb = (synth.bf16_bits(data[n]) for n in ("q", "k", "v"))
+    rng = np.random.default_rng(12345)
+
+    def draw(n):
+        b = rng.integers(0, len(L), n)
+        i = (rng.random(n) * L[b]).astype(np.int64)
+        h = rng.integers(0, w.Hq, n)
+        return np.stack([b, h, i], 1).astype(np.int32)
+
+    def run(rows):
+        t0 = time.perf_counter()
+        orc.attn_ragged_rows(qb, kb, vb, cu, cu, w.Hq, w.Hkv, w.scale, True, rows)
+        dt = time.perf_counter() - t0
+        fl = 4.0 * w.Dqk * float(np.sum(rows[:, 2].astype(np.int64) + 1))
+        return fl, dt
+
+    fl, dt = run(draw(256))
+    n = int(max(256, min(2_000_000, 256 * seconds / max(dt, 1e-3))))
+    rows = draw(n)
+    fl, dt = run(rows)
+    return fl / dt / 1e12, orc.num_threads(), (
+        f"{n} random (sequence, head, query) rows of the ragged prefill batch, "
+        f"{fl / 1e9:.1f} GFLOP in {dt:.1f} s")
+
+
+def oracle_decode_sample(data, seconds):
+    """The fp64 oracle on a random sample of (sequence, kv head) groups of the
+    decode batch (all G query heads of each group).  Returns (GB/s, threads, desc)."""
+    import oracle
+    import synth
+    w, L, table = data["w"], data["L"], data["table"]
+    orc = oracle.default()
+    qb = synth.bf16_bits(data["q"])
+    kb = synth.bf16_bits(data["kp"])
+    vb = kb if w.v_aliases_k else synth.bf16_bits(data["vp"])
+    kp = data["kp"]
+    ks = (kp.stride(0), kp.stride(2), kp.stride(1))
+    vs = ks if w.v_aliases_k else (data["vp"].stride(0), data["vp"].stride(2), data["vp"].stride(1))
+    G = w.Hq // w.Hkv
+    rng = np.random.default_rng(54321)
+
+    def run(ngroups):
+        b = rng.integers(0, w.B, ngroups)
+        g = rng.integers(0, w.Hkv, ngroups)
+        rows = np.array([(bb, gg * G + j) for bb, gg in zip(b, g) for j in range(G)], dtype=np.int32)
+        t0 = time.perf_counter()
+        orc.attn_paged_rows(qb, kb, vb, table, L.astype(np.int32), w.page_size, w.Hq, w.Hkv, w.Dqk,
+                            w.Dv, ks, vs, w.scale, rows)
+        dt = time.perf_counter() - t0
+        nb = float(np.sum(L[b])) * (w.Dqk if w.v_aliases_k else w.Dqk + w.Dv) * 2
+        return nb, dt, len(rows)
+
+    nb, dt, _ = run(4)
+    n = int(max(4, min(100_000, 4 * seconds / max(dt, 1e-3))))
+    nb, dt, nrows = run(n)
+    return nb / dt / 1e9, orc.num_threads(), (
+        f"{n} random (sequence, kv head) groups ({nrows} query rows) of the decode batch, "
+        f"{nb / 1e9:.2f} GB of K/V in {dt:.1f} s")
+
+
+def run_ours(args):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    dev = "cuda"
+    import ragged_scaled_dot_b200 as rsd
+    import synth
+    rsd.lib()  # fails loudly if the CUDA library is missing
+    peaks, peak_src = load_peaks()
+    num_sms = torch.cuda.get_device_properties(local).multi_processor_count
+
+    prefill, pdata = make_ragged_prefill(torch, rsd, synth, dev, rank * 1000)
+    decode, ddata = make_paged(torch, rsd, synth, dev, rank * 1000, "paged_decode", num_sms)
+    extras = []
+    if not args.no_extras:
+        extras.append(make_dense_prefill(torch, rsd, synth, dev, rank * 1000)[0])
+        mla, _ = make_paged(torch, rsd, synth, dev, rank * 1000, "mla_decode", num_sms)
+        extras.append(mla)
+    torch.cuda.synchronize()
+
+    results = {}
+    with ClockSampler(local) as clocks:
+        for part in [prefill, decode] + extras:
+            total_ms, per = time_part(torch, part, args.steps, args.warmup, dist, world)
+            results[part.name] = (total_ms, per)
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK, "device-side error during the bench"
+
+    def part_summary(part, bound):
+        total_ms, per = results[part.name]
+        ms = total_ms / args.steps
+        value = part.units * world / (total_ms / 1e3 / args.steps)
+        # dominant kernel: the part's launch sequence, timed per step on its stream
+        kern_ms = statistics.mean(per)
+        if bound == "tensor":
+            achieved = part.units / (kern_ms / 1e3)
+            peak = peaks["bf16_tflops"]
+            roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
+                    "peak_source": f"{peak_src} bf16_tflops (burst)"}
+        else:
+            achieved = part.units / (kern_ms / 1e3)
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_source": f"{peak_src} hbm_gbs"}
+        return value, ms, roof
+
+    p_val, p_ms, p_roof = part_summary(prefill, "tensor")
+    d_val, d_ms, d_roof = part_summary(decode, "hbm")
+
+    e2e = {}
+    for part in (prefill, decode):
+        ms, h2d, d2h = time_e2e(torch, part, max(1, min(3, args.steps)), dist)
+        e2e[part.name] = {"value": round(part.units * world / (ms / 1e3 / max(1, min(3, args.steps))), 3),
+                          "unit": part.unit, "h2d_bytes_per_step": int(h2d),
+                          "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / max(1, min(3, args.steps)), 3)}
+
+    cpu = {}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, c, desc = oracle_prefill_sample(pdata, args.cpu_seconds)
+        cpu["prefill"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": c, "kind": "oracle", "sample": desc}
+        v, c, desc = oracle_decode_sample(ddata, args.cpu_seconds)
+        cpu["decode"] = {"value": round(v, 4), "unit": "GB/s", "cores": c, "kind": "oracle", "sample": desc}
+
+    extra_out = {}
+    for part in extras:
+        bound = "tensor" if part.unit == "TFLOP/s" else "hbm"
+        v, ms, roof = part_summary(part, bound)
+        extra_out[part.name] = {"value": round(v, 2), "unit": part.unit, "ms_per_step": round(ms, 4),
+                                "roofline": roof, **part.info}
+        if part.name == "mla_decode":
+            tflops = part.info["flop_per_step"] / 1e12 / (ms / 1e3)
+            extra_out[part.name]["tflops"] = round(tflops, 2)
+            extra_out[part.name]["tensor_frac"] = round(tflops / peaks["bf16_tflops"], 4)
+            ridge_ms = max(part.units / peaks["hbm_gbs"], part.info["flop_per_step"] / 1e12 / peaks["bf16_tflops"]) * 1e3
+            extra_out[part.name]["roofline_frac_max_bound"] = round(ridge_ms / ms, 4)
+
+    if rank == 0:
+        ck = clocks.summary()
+        line = {
+            "metric": METRIC,
+            "value": round(p_val, 2),
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(p_ms, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic: N(0,1) bf16 Q/K/V, seeded lengths and page permutation",
+            "config": {"workload": "ragged THD causal prefill, 64 seqs U[128,8192], Hq/Hkv 32/8, "
+                                   "D 128, padded LSE (headline) + paged decode B 128 kv U[1024,32768] "
+                                   "page 64, Hq/Hkv 64/8, D 128, split-KV",
+                       "global_batch": prefill.info["B"] * world, "seq_len": prefill.info["max_seqlen"],
+                       "parallelism": f"replicas x{world} (independent batches)",
+                       "l2": "inputs larger than L2 (126 MB); no flush needed",
+                       "prefill": prefill.info, "decode": decode.info},
+            "roofline": p_roof,
+            "e2e": e2e["ragged_prefill"],
+            "decode": {"metric": "paged-decode KV GB/s", "value": round(d_val, 1), "unit": "GB/s",
+                       "ms_per_step": round(d_ms, 4), "roofline": d_roof, "e2e": e2e["paged_decode"]},
+            "extras": extra_out,
+            "gpu_launches": args.steps * (prefill.launches + decode.launches)
+                            + sum(args.steps * p.launches for p in extras),
+            "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"], "reasons": ck["reasons"],
+                       "samples": ck["samples"]},
+        }
+        if cpu:
+            line["cpu_baseline"] = dict(cpu["prefill"], decode=cpu["decode"])
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the fp64 oracle as it stands, on the host cores
+# --------------------------------------------------------------------------- #
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    import synth
+    w = synth.WORKLOADS["ragged_prefill"]
+    L = synth.uniform_lengths(w.B, *w.len_range, w.seed)
+    q, k, v, cu = synth.make_ragged(w, "cpu", lengths=L)
+    data = dict(q=q, k=k, v=v, cu=cu, L=L, w=w)
+    per_step = max(2.0, args.cpu_seconds / 4)
+    for _ in range(args.warmup if args.warmup < 2 else 1):
+        oracle_prefill_sample(data, 1.0)
+    vals, desc, cores = [], "", 1
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v_, cores, desc = oracle_prefill_sample(data, per_step)
+        vals.append(v_)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeds as our arm)",
+        "config": {"workload": "ragged THD causal prefill, 64 seqs U[128,8192], Hq/Hkv 32/8, D 128 "
+                               "(each step a bounded random row sample)"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del torch
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,216 @@
+/*
+ * b2attn.h -- C ABI of libb2attn.so: forward scaled-dot-product attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ *   O = softmax(scale * Q K^T + mask) V,   LSE = rowmax + ln(rowsum)   (fp32)
+ *
+ * in three layouts: dense BSHD, ragged/packed THD addressed through offset
+ * tables, and paged KV with split-KV partials merged by their LSE.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  Q, K, V and
+ *    O are bf16 (passed as void*); LSE and split partials are fp32.  Stats are
+ *    FP32 only ("cuDNN Frontend v1.28.0 release notes", "Updates to Graph API /
+ *    SDPA": Stats must be FP32).
+ *  - LSE is the natural log: rowmax + ln(rowsum) ("cuDNN Frontend v1.30.0
+ *    Release Notes", "New: stats_use_log2 -- LSE in base 2").  A query row that
+ *    sees no key gets O = 0 and LSE = -inf ("cuDNN Frontend v1.32.0 Release
+ *    Notes", "New: Rubin triangle operations").
+ *  - Strides are int64 ELEMENT counts, and the head dimension is always
+ *    contiguous (stride 1).  Every stride and the base pointer of Q, K, V and O
+ *    must be 16-byte aligned (a multiple of 8 elements); 64-bit addressing
+ *    throughout ("cuDNN Frontend v1.30.0 Release Notes", "New: prepared
+ *    launches", int64 stride leaves).
+ *  - `scale` is taken as given, 0 and negative values included ("cuDNN Frontend
+ *    v1.31.0 Release Notes", "Compatibility and numerical behavior": an explicit
+ *    zero is preserved).  It must be finite.
+ *  - GQA/MQA: query head h reads key/value head h / (Hq / Hkv); Hq must be a
+ *    multiple of Hkv ("cuDNN Frontend v1.30.0 Release Notes", "New: decode
+ *    tiles").
+ *  - Causal masking is bottom-right aligned per sequence: key j is visible to
+ *    query i of a sequence with Lq queries and Lkv keys iff j <= i + Lkv - Lq
+ *    ("cuDNN Frontend v1.28.0 release notes", "Masking, splitting, and
+ *    heuristics").
+ *  - The library owns no device memory, allocates none, and never blocks the
+ *    host: every entry point validates its arguments on the host, enqueues its
+ *    kernels on `stream` (a cudaStream_t passed as void*, NULL = legacy default
+ *    stream) and returns ("cuDNN Frontend v1.30.0 Release Notes", "Graph API,
+ *    Python API, and other operations": the graph API owns no device memory
+ *    and never blocks the host).  No entry point reads device memory back to
+ *    the host, so every call can be captured in a CUDA graph ("cuDNN Frontend
+ *    v1.28.0 release notes", "Ragged / THD, with zero host reads").
+ *  - Scratch space is caller-provided; a missing or undersized workspace is
+ *    rejected before launch ("cuDNN Frontend v1.31.0 Release Notes",
+ *    "Compatibility and numerical behavior": split-attention calls require
+ *    caller workspace).
+ *  - Return value: ATTN_OK or an error status.  Errors found on the host are
+ *    returned before anything is enqueued.  Conditions only the device can see
+ *    (inconsistent offset tables or lengths, out-of-range page ids, a bounded
+ *    wait that ran out) are recorded in a device-side status word that
+ *    attn_get_device_error() reads; the kernels never trap.
+ *  - Inputs are supported for Dqk, Dv in {64, 128} (prefill and decode) and
+ *    Dqk = 576, Dv = 512 (absorbed-MLA decode); other shapes are declined with
+ *    ATTN_ERR_UNSUPPORTED, never computed wrongly.
+ */
+#ifndef B2ATTN_H
+#define B2ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define ATTN_OK                  0
+#define ATTN_ERR_INVALID_ARG     1  /* a pointer, size, stride or alignment is invalid */
+#define ATTN_ERR_UNSUPPORTED     2  /* valid, but a shape this library declines      */
+#define ATTN_ERR_WORKSPACE       3  /* workspace missing or smaller than required     */
+#define ATTN_ERR_LAUNCH          4  /* a kernel launch failed (cudaGetLastError)      */
+#define ATTN_ERR_DEVICE_TIMEOUT  5  /* device: a bounded wait ran out                 */
+#define ATTN_ERR_DEVICE_INPUT    6  /* device: offsets / lengths / page ids invalid   */
+#define ATTN_ERR_CUDA            7  /* a CUDA runtime or driver call failed           */
+
+/* LSE layouts of attn_fwd_ragged. */
+#define ATTN_LSE_PADDED_BSH  0  /* [B, max_seqlen_q, Hq]; rows past a sequence's
+                                   length are set to -inf by the library on the
+                                   launch stream ("cuDNN Frontend v1.30.0 Release
+                                   Notes", "New: the FlashInfer serving path runs
+                                   on FROST": per-batch padded Stats seeded -inf) */
+#define ATTN_LSE_PACKED_TH   1  /* token-major [total_q, Hq]                    */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *attn_status_string(int status);
+
+/*
+ * Dense BSHD forward.
+ *   q: [B, Sq, Hq, Dqk]   k: [B, Skv, Hkv, Dqk]   v: [B, Skv, Hkv, Dv]
+ *   o: [B, Sq, Hq, Dv]    lse (nullable): fp32 [B, Hq, Sq], contiguous.
+ * x_strides[3] are the (batch, seq, head) element strides of each tensor, so
+ * strided views (e.g. slices of a fused QKV projection) are read in place
+ * ("cuDNN Frontend v1.30.0 Release Notes", "New: prepared launches": dense
+ * forward reads strided Q/K/V/O zero-copy).  Needs no workspace.
+ */
+int attn_fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
+                   int B, int Sq, int Skv, int Hq, int Hkv, int Dqk, int Dv,
+                   const int64_t q_strides[3], const int64_t k_strides[3],
+                   const int64_t v_strides[3], const int64_t o_strides[3],
+                   float scale, int causal, void *stream);
+
+/*
+ * Ragged / packed THD forward.
+ * Sequence b owns query tokens [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key /
+ * value tokens [cu_seqlens_kv[b], cu_seqlens_kv[b+1]); both tables are DEVICE
+ * int32 arrays of B+1 nondecreasing prefix sums starting at 0 ("cuDNN Frontend
+ * v1.28.0 release notes", "Ragged / THD, with zero host reads"; "cuDNN
+ * Frontend v1.30.0 Release Notes": the THD gate is over (H, S, D), the batch
+ * stride is never read).
+ *   q: element (t, h, d) at q[t*q_strides[0] + h*q_strides[1] + d]; same for
+ *   k, v, o with their own (token, head) strides.
+ * max_seqlen_q / max_seqlen_kv bound every sequence's length and total_q /
+ * total_kv bound the packed token counts; these host-declared capacities size
+ * the launch and the TMA bounds, so no token past total_q / total_kv is ever
+ * read or written ("cuDNN Frontend v1.28.0 release notes", "Updates to Graph
+ * API / SDPA": max_total_seq_len_q / _kv).  A device table that breaks them
+ * sets ATTN_ERR_DEVICE_INPUT and the offending sequences are skipped.
+ * lse (nullable): layout per lse_layout (ATTN_LSE_PADDED_BSH or _PACKED_TH).
+ * workspace: device scratch of at least attn_fwd_ragged_workspace_size(...)
+ * bytes, 256-byte aligned; it holds the device-built work list.
+ */
+int attn_fwd_ragged(const void *q, const void *k, const void *v, void *o, float *lse,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv,
+                    int B, int max_seqlen_q, int max_seqlen_kv,
+                    int64_t total_q, int64_t total_kv,
+                    int Hq, int Hkv, int Dqk, int Dv,
+                    const int64_t q_strides[2], const int64_t k_strides[2],
+                    const int64_t v_strides[2], const int64_t o_strides[2],
+                    int lse_layout, float scale, int causal,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes attn_fwd_ragged needs for these declared capacities. */
+size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q,
+                                      int Hq, int Hkv);
+
+/*
+ * Paged-KV decode forward: one query token per sequence, attending to all of
+ * its kv_lens[b] cached keys ("cuDNN Frontend v1.31.0 Release Notes", "SDPA:
+ * paged KV, split-KV, and engine selection").
+ *   q: [B, Hq, Dqk] with (batch, head) element strides q_strides[2].
+ *   o: [B, Hq, Dv]  with (batch, head) element strides o_strides[2].
+ *   lse (nullable): fp32 [B, Hq] contiguous.
+ *   k_pool / v_pool: pools of num_pages fixed-size pages; element
+ *   (page, slot, head, d) at pool[page*s[0] + slot*s[1] + head*s[2] + d] with
+ *   s = k_pool_strides / v_pool_strides, so K and V may have different
+ *   layouts.  Logical key t of sequence b is slot t % page_size of page
+ *   page_table[b*page_table_stride + t / page_size] (DEVICE int32).
+ *   Absorbed MLA: pass v_pool == k_pool with Dv < Dqk; V is then the first Dv
+ *   columns of each K row ("cuDNN Frontend v1.32.0 Release Notes", "SDPA:
+ *   wider native forward support": Q/K576, V512, absorbed-MLA cache layouts).
+ *   Each page-table row holds at least ceil(max_kv_len / page_size) entries.
+ *   kv_lens: DEVICE int32 [B], each in [0, max_kv_len]; page ids must lie in
+ *   [0, num_pages).  Violations set ATTN_ERR_DEVICE_INPUT on the device.
+ * Split-KV: each sequence's pages are cut into num_splits ranges of
+ * ceil(n_pages / num_splits) consecutive pages; num_splits > 1 writes fp32
+ * partial O and LSE into the workspace and merges them as attn_split_merge
+ * does.  workspace: >= attn_fwd_paged_workspace_size(...) bytes, 256-byte
+ * aligned (may be NULL when num_splits == 1).
+ */
+int attn_fwd_paged(const void *q, const void *k_pool, const void *v_pool, void *o,
+                   float *lse, const int32_t *page_table, int64_t page_table_stride,
+                   const int32_t *kv_lens, int B, int Hq, int Hkv, int Dqk, int Dv,
+                   int page_size, int64_t num_pages, int max_kv_len,
+                   const int64_t q_strides[2], const int64_t o_strides[2],
+                   const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
+                   float scale, int num_splits,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1). */
+size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits);
+
+/*
+ * A split count for attn_fwd_paged: enough (batch, head, split) blocks to keep
+ * num_sms SMs busy through the tail of uneven lengths, while the fp32 partials
+ * stay a small fraction of the KV bytes streamed.  Host-only arithmetic.
+ */
+int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len,
+                              int page_size, int num_sms);
+
+/*
+ * Split-KV merge by LSE, over R rows (R = B * Hq for decode):
+ *   LSE_r = ln sum_s exp(lse_part[s][r]),   O_r = sum_s exp(lse_part[s][r] - LSE_r) * o_part[s][r][:]
+ * Partials with lse = -inf (splits without keys) are ignored; a row whose
+ * partials are all -inf gets O = 0, LSE = -inf ("cuDNN Frontend v1.28.0 release
+ * notes", "Masking, splitting, and heuristics"; "cuDNN Frontend v1.30.0
+ * Release Notes", stats_use_log2 section on split partials).
+ *   o_part: fp32 [num_splits][R][Dv], lse_part: fp32 [num_splits][R] (contiguous)
+ *   o: bf16, row r at o + r*o_row_stride (elements);  lse (nullable): fp32 [R].
+ */
+int attn_split_merge(const float *o_part, const float *lse_part, int num_splits,
+                     int64_t R, int Dv, void *o, int64_t o_row_stride, float *lse,
+                     void *stream);
+
+/*
+ * Synchronizes `stream`, returns the device-side status word (ATTN_OK,
+ * ATTN_ERR_DEVICE_TIMEOUT or ATTN_ERR_DEVICE_INPUT; the first error recorded
+ * since the last call) for the current device, and clears it.  This is the one
+ * entry point that blocks the host; it is a diagnostic, not part of the
+ * compute path.
+ */
+int attn_get_device_error(void *stream);
+
+/*
+ * Fault-free check of the bounded-wait machinery: launches one block that
+ * waits, with the library's bounded wait and a limit of timeout_ns
+ * nanoseconds, on a barrier nothing ever signals.  The wait runs out, the
+ * kernel records ATTN_ERR_DEVICE_TIMEOUT and returns; the context stays
+ * usable.  Returns the launch status.
+ */
+int attn_selftest_bounded_wait(uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B2ATTN_H */

@@ -1,0 +1,189 @@
+// aux_kernels.cuh -- device-side metadata for the ragged layout, the padded
+// LSE fill, the split-KV LSE merge and the bounded-wait self-test.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace b2 {
+
+// ---------------------------------------------------------------------------
+// Ragged work list, built on the device from the offset tables so the host
+// never reads them back ("cuDNN Frontend v1.28.0 release notes", "Ragged /
+// THD, with zero host reads").  One block:
+//   1. validate each sequence against the host-declared capacities;
+//   2. histogram the work items by cost (KV tiles to visit);
+//   3. counting-sort them longest first (LPT) into `items`.
+// Items of one (sequence, query tile) are adjacent, one per query-head group.
+// ---------------------------------------------------------------------------
+constexpr int kCostBuckets = 4096;
+
+__device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t* cu_kv, int b,
+                                              int max_sq, int max_skv, int64_t total_q,
+                                              int64_t total_kv) {
+    const int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_kv[b], k1 = cu_kv[b + 1];
+    const int lq = q1 - q0, lk = k1 - k0;
+    return q0 >= 0 && k0 >= 0 && lq >= 0 && lk >= 0 && lq <= max_sq && lk <= max_skv &&
+           (int64_t)q1 <= total_q && (int64_t)k1 <= total_kv;
+}
+
+__global__ void __launch_bounds__(1024) ragged_worklist_kernel(
+    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv, int B, int max_sq,
+    int max_skv, int64_t total_q, int64_t total_kv, int causal, int n_pairs, int heads_per_item,
+    int4* __restrict__ items, int* __restrict__ n_items_out, int max_tiles) {
+    __shared__ int hist[kCostBuckets];
+    __shared__ int n_tiles_sh;
+    for (int i = threadIdx.x; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
+    if (threadIdx.x == 0) {
+        n_tiles_sh = 0;
+        if (cu_q[0] != 0 || cu_kv[0] != 0) record_status(ATTN_ERR_DEVICE_INPUT);
+    }
+    __syncthreads();
+    // pass 1: validate + histogram of costs
+    int my_tiles = 0;
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        if (!ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv)) {
+            record_status(ATTN_ERR_DEVICE_INPUT);
+            continue;
+        }
+        const int lq = cu_q[b + 1] - cu_q[b], lk = cu_kv[b + 1] - cu_kv[b];
+        const int nqt = (lq + 127) >> 7;
+        for (int qt = 0; qt < nqt; ++qt) {
+            const int cost = min(prefill_n_kv(qt, lq, lk, causal), kCostBuckets - 1);
+            atomicAdd(&hist[cost], 1);
+        }
+        my_tiles += nqt;
+    }
+    atomicAdd(&n_tiles_sh, my_tiles);
+    __syncthreads();
+    // exclusive scan, highest cost first (single thread: 4096 buckets)
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int c = kCostBuckets - 1; c >= 0; --c) {
+            const int h = hist[c];
+            hist[c] = run;
+            run += h;
+        }
+        const int n = min(n_tiles_sh, max_tiles);
+        if (n_tiles_sh > max_tiles) record_status(ATTN_ERR_DEVICE_INPUT);
+        *n_items_out = n * n_pairs;
+    }
+    __syncthreads();
+    // pass 2: scatter
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        if (!ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv)) continue;
+        const int lq = cu_q[b + 1] - cu_q[b], lk = cu_kv[b + 1] - cu_kv[b];
+        const int nqt = (lq + 127) >> 7;
+        for (int qt = 0; qt < nqt; ++qt) {
+            const int cost = prefill_n_kv(qt, lq, lk, causal);
+            const int pos = atomicAdd(&hist[min(cost, kCostBuckets - 1)], 1);
+            if (pos >= max_tiles) continue;
+            for (int pr = 0; pr < n_pairs; ++pr)
+                items[(int64_t)pos * n_pairs + pr] = make_int4(b, qt, pr * heads_per_item, cost);
+        }
+    }
+}
+
+// Padded (b, s_max, h) LSE: rows at or past a sequence's length are -inf
+// ("cuDNN Frontend v1.30.0 Release Notes", "New: the FlashInfer serving path
+// runs on FROST": the padded Stats buffer is seeded with -inf on the launch
+// stream).  Rows inside a sequence are written by the prefill kernel.
+__global__ void lse_padded_fill_kernel(const int32_t* __restrict__ cu_q, int B, int smax, int Hq,
+                                       float* __restrict__ lse) {
+    const int64_t n = (int64_t)B * smax * Hq;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bs = i / Hq;
+        const int b = (int)(bs / smax);
+        const int s = (int)(bs - (int64_t)b * smax);
+        int lq = cu_q[b + 1] - cu_q[b];
+        lq = max(0, min(lq, smax));
+        if (s >= lq) lse[i] = -INFINITY;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Split-KV merge by LSE.  One warp per row r:
+//   M = max_s lse_s;  w_s = exp(lse_s - LSE) with LSE = M + ln sum_s exp(lse_s - M)
+//   O = sum_s w_s O_s.   All partials -inf -> O = 0, LSE = -inf.
+// Computed in the log2 domain: exp(x) = 2^(x log2 e).
+// ---------------------------------------------------------------------------
+template <int DV>
+__global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part,
+                                                          int S, int64_t R,
+                                                          __nv_bfloat16* __restrict__ o,
+                                                          int64_t o_row_stride,
+                                                          float* __restrict__ lse) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr int VEC = (DV % 128 == 0) ? 4 : 2;  // floats per vector access
+    constexpr int NV = DV / (32 * VEC);           // vector accesses per lane
+    static_assert(NV >= 1 && DV % (32 * VEC) == 0, "unsupported Dv");
+    const int64_t r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= R) return;
+    float M = -INFINITY;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, lse_part[(int64_t)s * R + r]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float acc[NV][VEC];
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[i][e] = 0.f;
+    float L = -INFINITY;
+    if (M != -INFINITY) {
+        float sum = 0.f;
+        for (int s = lane; s < S; s += 32) sum += ex2((lse_part[(int64_t)s * R + r] - M) * LOG2E);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        L = M + logf(sum);
+        for (int s = 0; s < S; ++s) {
+            const float ls = lse_part[(int64_t)s * R + r];
+            if (ls == -INFINITY) continue;
+            const float w = ex2((ls - L) * LOG2E);
+            const float* src = o_part + ((int64_t)s * R + r) * DV;
+#pragma unroll
+            for (int i = 0; i < NV; ++i) {
+                const int e0 = VEC * (lane + 32 * i);
+                if constexpr (VEC == 4) {
+                    const float4 v = __ldg(reinterpret_cast<const float4*>(src + e0));
+                    acc[i][0] += w * v.x; acc[i][1] += w * v.y;
+                    acc[i][2] += w * v.z; acc[i][3] += w * v.w;
+                } else {
+                    const float2 v = __ldg(reinterpret_cast<const float2*>(src + e0));
+                    acc[i][0] += w * v.x; acc[i][1] += w * v.y;
+                }
+            }
+        }
+    }
+    __nv_bfloat16* dst = o + r * o_row_stride;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e0 = VEC * (lane + 32 * i);
+        if constexpr (VEC == 4) {
+            uint2 w;
+            w.x = pack_bf16(acc[i][0], acc[i][1]);
+            w.y = pack_bf16(acc[i][2], acc[i][3]);
+            *reinterpret_cast<uint2*>(dst + e0) = w;
+        } else {
+            *reinterpret_cast<uint32_t*>(dst + e0) = pack_bf16(acc[i][0], acc[i][1]);
+        }
+    }
+    if (lse != nullptr && lane == 0) lse[r] = L;
+}
+
+// Bounded-wait self-test: waits on a barrier that nothing signals.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, (volatile int*)&abort_flag, limit_ns);
+    __syncthreads();
+}
+
+}  // namespace b2

@@ -1,0 +1,479 @@
+// b2attn.cu -- the C ABI of libb2attn.so (see include/b2attn.h): host-side
+// validation, TMA descriptor encoding and kernel launches.  Nothing here
+// allocates device memory, reads device memory back or synchronizes, except
+// attn_get_device_error(), which is a diagnostic.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "b2attn.h"
+#include "ptx.cuh"
+#include "prefill.cuh"
+#include "aux_kernels.cuh"
+#include "decode.cuh"
+
+namespace {
+
+using b2::DecodeParams;
+using b2::PrefillParams;
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxDevices = 64;
+
+// ---------------------------------------------------------------------------
+// Per-device one-time set-up: SM count and kernel shared-memory opt-ins.
+// ---------------------------------------------------------------------------
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int setup_device(int* dev_out, int* sms_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        if (g_encode == nullptr) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                fn == nullptr)
+                return ATTN_ERR_CUDA;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ATTN_ERR_CUDA;
+        cudaError_t e = cudaSuccess;
+        e = cudaFuncSetAttribute(b2::prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 b2::PrefillCfg<64>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::PrefillCfg<128>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::decode_gqa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::DecodeCfg<64>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::decode_gqa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::DecodeCfg<128>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::decode_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::MlaCfg<true>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::decode_mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::MlaCfg<false>::SMEM);
+        if (e != cudaSuccess) return ATTN_ERR_CUDA;
+        st.num_sms = sms;
+        st.ready = true;
+    }
+    *dev_out = dev;
+    *sms_out = st.num_sms;
+    return ATTN_OK;
+}
+
+// 4D bf16 tensor map with 128-byte swizzle.  dims/strides: innermost first;
+// strides in ELEMENTS for dims 1..3.  Box inner extent is 64 elements (128 B).
+int encode_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const int64_t strides_el[3],
+              const uint32_t box[4]) {
+    cuuint64_t gdim[4], gstr[3];
+    cuuint32_t bdim[4], estr[4] = {1, 1, 1, 1};
+    for (int i = 0; i < 4; ++i) {
+        if (dims[i] == 0 || dims[i] > (1ull << 32)) return ATTN_ERR_INVALID_ARG;
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+    }
+    for (int i = 0; i < 3; ++i) {
+        const int64_t bytes = strides_el[i] * 2;
+        if (bytes <= 0 || (bytes % 16) != 0 || bytes >= (int64_t(1) << 40)) return ATTN_ERR_INVALID_ARG;
+        gstr[i] = (cuuint64_t)bytes;
+    }
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim, gstr, bdim,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+
+// A stride for a tensor-map dimension of extent 1 (never stepped along).
+int64_t unit_dim_stride(int64_t a, int64_t b) { return round_up(a > b ? a : b, 8); }
+
+int ragged_max_tiles(int B, int max_sq, int64_t total_q) {
+    const int64_t by_total = total_q / 128 + B;
+    const int64_t by_max = (int64_t)B * ((max_sq + 127) / 128);
+    int64_t t = by_total < by_max ? by_total : by_max;
+    if (t > (int64_t)1 << 30) t = (int64_t)1 << 30;
+    return (int)t;
+}
+
+void pair_shape(int Hq, int Hkv, int* hpi, int* n_pairs) {
+    const int G = Hq / Hkv;
+    *hpi = (G % 2 == 0) ? 2 : 1;
+    *n_pairs = Hq / *hpi;
+}
+
+// Launches the prefill kernel for an already-filled PrefillParams.
+int launch_prefill(PrefillParams& pp, int D, int grid, cudaStream_t st) {
+    if (grid <= 0) return ATTN_OK;
+    if (D == 128)
+        b2::prefill_kernel<128><<<grid, 384, b2::PrefillCfg<128>::SMEM, st>>>(pp);
+    else
+        b2::prefill_kernel<64><<<grid, 384, b2::PrefillCfg<64>::SMEM, st>>>(pp);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG: invalid pointer, size, stride or alignment";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED: shape declined by this library";
+        case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE: workspace missing or too small";
+        case ATTN_ERR_LAUNCH: return "ATTN_ERR_LAUNCH: kernel launch failed";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+        case ATTN_ERR_DEVICE_INPUT: return "ATTN_ERR_DEVICE_INPUT: device offsets, lengths or page ids invalid";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: CUDA runtime or driver call failed";
+        default: return "unknown status";
+    }
+}
+
+// ------------------------------------------------------------------ dense
+int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv,
+                   int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[3], const int64_t k_strides[3],
+                   const int64_t v_strides[3], const int64_t o_strides[3], float scale, int causal,
+                   void* stream) {
+    if (B < 0 || Sq < 0 || Skv < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+    if (!q_strides || !k_strides || !v_strides || !o_strides) return ATTN_ERR_INVALID_ARG;
+    if (Dqk != Dv || (Dqk != 64 && Dqk != 128)) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || Sq == 0) return ATTN_OK;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (!stride_ok(q_strides[i]) || !stride_ok(k_strides[i]) || !stride_ok(v_strides[i]) ||
+            !stride_ok(o_strides[i]))
+            return ATTN_ERR_INVALID_ARG;
+    int dev, sms;
+    if (int e = setup_device(&dev, &sms)) return e;
+    const int D = Dqk;
+    PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    {
+        const uint32_t box[4] = {64, 1, 128, 1};
+        const uint64_t dq[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Sq, (uint64_t)B};
+        const int64_t sq[3] = {q_strides[2], q_strides[1], q_strides[0]};
+        if (encode_4d(&pp.tm_q, q, dq, sq, box)) return ATTN_ERR_INVALID_ARG;
+        const uint64_t dkv[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)(Skv > 0 ? Skv : 1), (uint64_t)B};
+        const int64_t sk[3] = {k_strides[2], k_strides[1], k_strides[0]};
+        const int64_t sv[3] = {v_strides[2], v_strides[1], v_strides[0]};
+        if (encode_4d(&pp.tm_k, k, dkv, sk, box)) return ATTN_ERR_INVALID_ARG;
+        if (encode_4d(&pp.tm_v, v, dkv, sv, box)) return ATTN_ERR_INVALID_ARG;
+    }
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    pp.mode = 0;
+    pp.B = B;
+    pp.Hq = Hq;
+    pp.Hkv = Hkv;
+    pp.G = Hq / Hkv;
+    pp.heads_per_item = hpi;
+    pp.n_pairs = n_pairs;
+    pp.Sq = Sq;
+    pp.Skv = Skv;
+    pp.n_qtiles = (Sq + 127) / 128;
+    const int64_t n_items = (int64_t)B * n_pairs * pp.n_qtiles;
+    if (n_items >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
+    pp.n_items = (int)n_items;
+    pp.o = static_cast<__nv_bfloat16*>(o);
+    pp.o_bs = o_strides[0];
+    pp.o_ts = o_strides[1];
+    pp.o_hs = o_strides[2];
+    pp.lse = lse;
+    pp.lse_layout = 0;
+    pp.scale_log2 = scale * kLog2e;
+    pp.causal = causal;
+    const int grid = (int)(n_items < sms ? n_items : sms);
+    return launch_prefill(pp, D, grid, static_cast<cudaStream_t>(stream));
+}
+
+// ----------------------------------------------------------------- ragged
+size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seqlen_q < 0 || total_q < 0) return 0;
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int64_t tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
+    return (size_t)(256 + tiles * n_pairs * 16);
+}
+
+int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_kv, int B, int max_seqlen_q, int max_seqlen_kv, int64_t total_q,
+                    int64_t total_kv, int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[2],
+                    const int64_t k_strides[2], const int64_t v_strides[2], const int64_t o_strides[2],
+                    int lse_layout, float scale, int causal, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    if (B < 0 || max_seqlen_q < 0 || max_seqlen_kv < 0 || total_q < 0 || total_kv < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+    if (lse_layout != ATTN_LSE_PADDED_BSH && lse_layout != ATTN_LSE_PACKED_TH) return ATTN_ERR_INVALID_ARG;
+    if (!q_strides || !k_strides || !v_strides || !o_strides) return ATTN_ERR_INVALID_ARG;
+    if (Dqk != Dv || (Dqk != 64 && Dqk != 128)) return ATTN_ERR_UNSUPPORTED;
+    if (total_q >= ((int64_t)1 << 31) || total_kv >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+    if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_kv) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 2; ++i)
+        if (!stride_ok(q_strides[i]) || !stride_ok(k_strides[i]) || !stride_ok(v_strides[i]) ||
+            !stride_ok(o_strides[i]))
+            return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
+    if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
+    int dev, sms;
+    if (int e = setup_device(&dev, &sms)) return e;
+    const int D = Dqk;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    {
+        const uint32_t box[4] = {64, 1, 128, 1};
+        const uint64_t dq[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)total_q, 1};
+        const int64_t sq[3] = {q_strides[1], q_strides[0], unit_dim_stride(q_strides[0] * total_q, 8)};
+        if (encode_4d(&pp.tm_q, q, dq, sq, box)) return ATTN_ERR_INVALID_ARG;
+        const uint64_t dkv[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)(total_kv > 0 ? total_kv : 1), 1};
+        const int64_t sk[3] = {k_strides[1], k_strides[0], unit_dim_stride(k_strides[0] * total_kv, 8)};
+        const int64_t sv[3] = {v_strides[1], v_strides[0], unit_dim_stride(v_strides[0] * total_kv, 8)};
+        if (encode_4d(&pp.tm_k, k, dkv, sk, box)) return ATTN_ERR_INVALID_ARG;
+        if (encode_4d(&pp.tm_v, v, dkv, sv, box)) return ATTN_ERR_INVALID_ARG;
+    }
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
+    int* n_items_dev = static_cast<int*>(workspace);
+    int4* items = reinterpret_cast<int4*>(static_cast<char*>(workspace) + 256);
+
+    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv,
+                                                   total_q, total_kv, causal, n_pairs, hpi, items, n_items_dev,
+                                                   max_tiles);
+    if (int e = launch_status()) return e;
+    if (lse != nullptr && lse_layout == ATTN_LSE_PADDED_BSH) {
+        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
+        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
+        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
+        if (int e = launch_status()) return e;
+    }
+    pp.mode = 1;
+    pp.B = B;
+    pp.Hq = Hq;
+    pp.Hkv = Hkv;
+    pp.G = Hq / Hkv;
+    pp.heads_per_item = hpi;
+    pp.n_pairs = n_pairs;
+    pp.cu_q = cu_seqlens_q;
+    pp.cu_kv = cu_seqlens_kv;
+    pp.items = items;
+    pp.n_items_dev = n_items_dev;
+    pp.o = static_cast<__nv_bfloat16*>(o);
+    pp.o_bs = 0;
+    pp.o_ts = o_strides[0];
+    pp.o_hs = o_strides[1];
+    pp.lse = lse;
+    pp.lse_layout = (lse_layout == ATTN_LSE_PADDED_BSH) ? 1 : 2;
+    pp.lse_smax = max_seqlen_q;
+    pp.scale_log2 = scale * kLog2e;
+    pp.causal = causal;
+    const int64_t items_max = (int64_t)max_tiles * n_pairs;
+    const int grid = (int)(items_max < sms ? items_max : sms);
+    return launch_prefill(pp, D, grid, st);
+}
+
+// ------------------------------------------------------------------ paged
+size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits) {
+    if (B <= 0 || Hq <= 0 || Dv <= 0 || num_splits <= 1) return 0;
+    const int64_t R = (int64_t)B * Hq;
+    return (size_t)(round_up(R * num_splits * Dv * 4, 256) + round_up(R * num_splits * 4, 256));
+}
+
+int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len, int page_size,
+                              int num_sms) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_kv_len <= 0 || page_size <= 0 || num_sms <= 0) return 1;
+    const bool mla = (Dqk == 576);
+    const int64_t ctas_per_split = mla ? (Hq / 64 > 0 ? Hq / 64 : 1) * (int64_t)B : (int64_t)Hkv * B;
+    const int64_t slots = (int64_t)num_sms * (mla ? 1 : 2);
+    int64_t s_balance = (8 * slots + ctas_per_split - 1) / ctas_per_split;
+    // keep the fp32 partials (written + read) under ~5% of the KV bytes streamed
+    const double kv_bytes = 0.5 * (double)max_kv_len * Hkv * (double)(mla ? Dqk : Dqk + Dv) * 2.0;
+    const double part_bytes_per_split = (double)Hq * Dv * 8.0;
+    int64_t s_traffic = (int64_t)(0.05 * kv_bytes / part_bytes_per_split);
+    int64_t s = s_balance < s_traffic ? s_balance : s_traffic;
+    const int64_t max_pages = (max_kv_len + page_size - 1) / page_size;
+    if (s > max_pages) s = max_pages;
+    if (s > 64) s = 64;
+    if (s < 1) s = 1;
+    return (int)s;
+}
+
+int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
+                   const int32_t* page_table, int64_t page_table_stride, const int32_t* kv_lens, int B, int Hq,
+                   int Hkv, int Dqk, int Dv, int page_size, int64_t num_pages, int max_kv_len,
+                   const int64_t q_strides[2], const int64_t o_strides[2], const int64_t k_pool_strides[3],
+                   const int64_t v_pool_strides[3], float scale, int num_splits, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_kv_len < 0 || num_pages < 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || num_splits < 1 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
+    if (!q_strides || !o_strides || !k_pool_strides || !v_pool_strides) return ATTN_ERR_INVALID_ARG;
+    if (page_size <= 0 || page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    const bool mla = (Dqk == 576 && Dv == 512);
+    const bool gqa = (Dqk == Dv && (Dqk == 64 || Dqk == 128) && G <= 16);
+    if (!mla && !gqa) return ATTN_ERR_UNSUPPORTED;
+    if (mla && (Hkv != 1 || Hq % 64 != 0)) return ATTN_ERR_UNSUPPORTED;
+    // a 64-key chunk is whole pages, or a page is whole chunks
+    if (!(page_size % 64 == 0 || (64 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
+    if (mla && !(page_size % 32 == 0 || (32 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535 || num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0) return ATTN_OK;
+    if (!q || !k_pool || !v_pool || !o || !page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (num_pages == 0) return ATTN_ERR_INVALID_ARG;
+    // every row of the page table must cover max_kv_len keys
+    if (B > 1 && page_table_stride < ((int64_t)max_kv_len + page_size - 1) / page_size) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 2; ++i)
+        if (!stride_ok(q_strides[i]) || !stride_ok(o_strides[i])) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (!stride_ok(k_pool_strides[i]) || !stride_ok(v_pool_strides[i])) return ATTN_ERR_INVALID_ARG;
+    if (num_splits > 1) {
+        const size_t need = attn_fwd_paged_workspace_size(B, Hq, Dv, num_splits);
+        if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
+    }
+    int dev, sms;
+    if (int e = setup_device(&dev, &sms)) return e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool alias = mla && (v_pool == k_pool) && std::memcmp(k_pool_strides, v_pool_strides, 3 * sizeof(int64_t)) == 0;
+
+    DecodeParams dp;
+    std::memset(&dp, 0, sizeof(dp));
+    // rows per TMA box: one page, at most one chunk (64 keys GQA, 32 keys MLA)
+    const int chunk_keys = mla ? 32 : 64;
+    const int box_rows = page_size < chunk_keys ? page_size : chunk_keys;
+    {
+        const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
+        const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
+        const int64_t sk[3] = {k_pool_strides[1], k_pool_strides[2], k_pool_strides[0]};
+        if (encode_4d(&dp.tm_k, k_pool, dk, sk, box)) return ATTN_ERR_INVALID_ARG;
+        const uint64_t dv[4] = {(uint64_t)Dv, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
+        const int64_t sv[3] = {v_pool_strides[1], v_pool_strides[2], v_pool_strides[0]};
+        if (encode_4d(&dp.tm_v, v_pool, dv, sv, box)) return ATTN_ERR_INVALID_ARG;
+        if (mla) {
+            const uint32_t qbox[4] = {64, 64, 1, 1};
+            const uint64_t dq[4] = {(uint64_t)Dqk, (uint64_t)Hq, (uint64_t)B, 1};
+            const int64_t sq[3] = {q_strides[1], q_strides[0], unit_dim_stride(q_strides[0] * B, 8)};
+            if (encode_4d(&dp.tm_q, q, dq, sq, qbox)) return ATTN_ERR_INVALID_ARG;
+        }
+    }
+    dp.q = static_cast<const __nv_bfloat16*>(q);
+    dp.q_bs = q_strides[0];
+    dp.q_hs = q_strides[1];
+    dp.page_table = page_table;
+    dp.pt_stride = page_table_stride;
+    dp.kv_lens = kv_lens;
+    dp.B = B;
+    dp.Hq = Hq;
+    dp.Hkv = Hkv;
+    dp.G = G;
+    dp.page_size = page_size;
+    dp.box_rows = box_rows;
+    dp.num_pages = num_pages;
+    dp.max_kv_len = max_kv_len;
+    dp.num_splits = num_splits;
+    dp.scale_log2 = scale * kLog2e;
+    dp.o = static_cast<__nv_bfloat16*>(o);
+    dp.o_bs = o_strides[0];
+    dp.o_hs = o_strides[1];
+    dp.lse = lse;
+    const int64_t R = (int64_t)B * Hq;
+    if (num_splits > 1) {
+        dp.o_part = static_cast<float*>(workspace);
+        dp.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                               round_up(R * num_splits * Dv * 4, 256));
+    }
+    if (mla) {
+        dim3 grid(num_splits, Hq / 64, B);
+        if (alias)
+            b2::decode_mla_kernel<true><<<grid, 288, b2::MlaCfg<true>::SMEM, st>>>(dp);
+        else
+            b2::decode_mla_kernel<false><<<grid, 288, b2::MlaCfg<false>::SMEM, st>>>(dp);
+    } else {
+        dim3 grid(num_splits, Hkv, B);
+        if (Dqk == 128)
+            b2::decode_gqa_kernel<128><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+        else
+            b2::decode_gqa_kernel<64><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+    }
+    if (int e = launch_status()) return e;
+    if (num_splits > 1) {
+        // O rows are (b, h); merge writes row r = b*Hq + h at o + b*o_bs + h*o_hs.
+        if (o_strides[0] != (int64_t)Hq * o_strides[1]) return ATTN_ERR_UNSUPPORTED;
+        return attn_split_merge(dp.o_part, dp.lse_part, num_splits, R, Dv, o, o_strides[1], lse, stream);
+    }
+    return ATTN_OK;
+}
+
+// ------------------------------------------------------------------ merge
+int attn_split_merge(const float* o_part, const float* lse_part, int num_splits, int64_t R, int Dv, void* o,
+                     int64_t o_row_stride, float* lse, void* stream) {
+    if (num_splits < 1 || R < 0 || o_row_stride < Dv) return ATTN_ERR_INVALID_ARG;
+    if (Dv != 64 && Dv != 128 && Dv != 512) return ATTN_ERR_UNSUPPORTED;
+    if (R == 0) return ATTN_OK;
+    if (!o_part || !lse_part || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(o_part) || (reinterpret_cast<uintptr_t>(o) & 7u) || (o_row_stride % 4) != 0)
+        return ATTN_ERR_INVALID_ARG;
+    int dev, sms;
+    if (int e = setup_device(&dev, &sms)) return e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t blocks = (R + 7) / 8;
+    if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+    if (Dv == 64)
+        b2::split_merge_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(o_part, lse_part, num_splits, R, ob, o_row_stride, lse);
+    else if (Dv == 128)
+        b2::split_merge_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(o_part, lse_part, num_splits, R, ob, o_row_stride, lse);
+    else
+        b2::split_merge_kernel<512><<<(unsigned)blocks, 256, 0, st>>>(o_part, lse_part, num_splits, R, ob, o_row_stride, lse);
+    return launch_status();
+}
+
+// ------------------------------------------------------------- diagnostics
+int attn_get_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, b2::g_device_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(b2::g_device_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return v;
+}
+
+int attn_selftest_bounded_wait(uint64_t timeout_ns, void* stream) {
+    b2::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns);
+    return launch_status();
+}
+
+}  // extern "C"

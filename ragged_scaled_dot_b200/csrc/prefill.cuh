@@ -1,0 +1,438 @@
+// prefill.cuh -- forward attention prefill on tcgen05 tensor cores (sm_100a).
+//
+// One persistent CTA per SM walks a longest-first work list.  A work item is
+// (sequence b, query tile of 128 rows, up to two query heads of one GQA group):
+// the two heads share every K/V tile, so each K/V byte brought on chip feeds
+// two 128x128 score tiles ("cuDNN Frontend v1.30.0 Release Notes", "New:
+// decode tiles", GQA packing; the grouping here is our own).
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q tiles of the item, then K(j), V(j) into a ring.
+//   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit.
+//   warps 4-7   softmax for slot 0 (query head h0), one TMEM lane (row) each.
+//   warps 8-11  softmax for slot 1 (query head h0 + 1).
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
+// P (bf16) overwrites the first 64 columns of its S tile and feeds the PV MMA
+// straight from TMEM.
+//
+// MMA order per KV tile j (FA4-style ping-pong between the two slots):
+//   PV0(j) QK0(j+1) PV1(j) QK1(j+1)
+// so the tensor core computes one slot's MMAs while the other slot's softmax
+// runs.  The softmax keeps the running maximum m in the log2 domain with the
+// scale folded in ("cuDNN Frontend v1.30.0 Release Notes", stats_use_log2
+// section: the prefill kernels keep the softmax in the log2 domain) and only
+// rescales O when the maximum grows by more than 8 (P stays <= 2^8).
+//
+// Masking: bottom-right causal per sequence and ragged tails are applied by
+// select (-inf), never by multiplication, so values past a sequence's end can
+// not poison a row through 0 * NaN ("cuDNN Frontend v1.28.0 release notes",
+// "Updates to Graph API / SDPA", max_total_seq_len).  Fully masked KV tiles
+// past the causal diagonal are never loaded.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace b2 {
+
+struct PrefillParams {
+    CUtensorMap tm_q;  // 4D (d, head, token, batch), 128B swizzle, box (64, 1, 128, 1)
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;
+    int mode;  // 0 dense, 1 ragged
+    int B, Hq, Hkv, G;
+    int heads_per_item;  // 2 when G is even, else 1
+    int n_pairs;         // Hq / heads_per_item
+    int Sq, Skv;         // dense
+    int n_qtiles;        // dense: ceil(Sq / 128)
+    int n_items;         // dense: number of work items
+    const int32_t* cu_q;
+    const int32_t* cu_kv;
+    const int4* items;     // ragged: work list {b, qtile, h0, cost}
+    const int* n_items_dev;  // ragged: its length
+    __nv_bfloat16* o;
+    int64_t o_bs, o_ts, o_hs;  // element strides (batch, token, head)
+    float* lse;
+    int lse_layout;  // 0 dense [B,Hq,Sq], 1 padded [B,smax,Hq], 2 packed [T,Hq]
+    int lse_smax;
+    float scale_log2;
+    int causal;
+};
+
+struct PrefillItem {
+    int b, qt, h0, nh;
+    int q_tok0;      // token coordinate of row 0 (dense: inside the batch)
+    int kv_tok0;     // token coordinate of key 0
+    int batch;       // batch coordinate (dense) or 0
+    int Lq, Lkv;
+    int n_kv;        // KV tiles to visit
+};
+
+__device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal) {
+    const int total = (Lkv + 127) >> 7;
+    if (!causal) return total;
+    const int rows = min(128, Lq - qt * 128);
+    const long long kmax = (long long)qt * 128 + rows - 1 + (long long)(Lkv - Lq);
+    if (kmax < 0) return 0;
+    return (int)min((long long)total, (kmax >> 7) + 1);
+}
+
+__device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx, PrefillItem& it) {
+    if (p.mode == 0) {
+        const int per_tile = p.B * p.n_pairs;
+        const int q = idx / per_tile;
+        const int rem = idx - q * per_tile;
+        it.qt = p.causal ? (p.n_qtiles - 1 - q) : q;  // longest (latest) tiles first
+        it.b = rem / p.n_pairs;
+        it.h0 = (rem - it.b * p.n_pairs) * p.heads_per_item;
+        it.q_tok0 = it.qt * 128;
+        it.kv_tok0 = 0;
+        it.batch = it.b;
+        it.Lq = p.Sq;
+        it.Lkv = p.Skv;
+    } else {
+        const int4 w = p.items[idx];
+        it.b = w.x;
+        it.qt = w.y;
+        it.h0 = w.z;
+        const int q0 = __ldg(p.cu_q + it.b), q1 = __ldg(p.cu_q + it.b + 1);
+        const int k0 = __ldg(p.cu_kv + it.b), k1 = __ldg(p.cu_kv + it.b + 1);
+        it.Lq = q1 - q0;
+        it.Lkv = k1 - k0;
+        it.q_tok0 = q0 + it.qt * 128;
+        it.kv_tok0 = k0;
+        it.batch = 0;
+    }
+    it.nh = p.heads_per_item;
+    it.n_kv = prefill_n_kv(it.qt, it.Lq, it.Lkv, p.causal);
+}
+
+template <int D>
+struct PrefillCfg {
+    static constexpr int HALVES = D / 64;
+    static constexpr uint32_t TILE = HALVES * 16384u;  // one 128-row bf16 tile
+    static constexpr int NST = (D == 128) ? 5 : 8;     // K/V ring depth
+    static constexpr uint32_t BAR_OFF = (2 + NST) * TILE;
+    static constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+};
+
+template <int D>
+__global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+    using C = PrefillCfg<D>;
+    constexpr int NST = C::NST;
+    constexpr uint32_t TILE = C::TILE;
+    constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sb - raw);
+    const uint32_t sQ = sb;
+    const uint32_t sKV = sb + 2 * TILE;
+    const uint32_t sBar = sb + C::BAR_OFF;
+    auto full_bar = [&](int i) { return sBar + 8u * i; };
+    auto empty_bar = [&](int i) { return sBar + 8u * (NST + i); };
+    const uint32_t b_qfull = sBar + 16u * NST;
+    const uint32_t b_qempty = b_qfull + 8;
+    const uint32_t b_sfull0 = b_qfull + 16;   // + 8*slot
+    const uint32_t b_pready0 = b_qfull + 32;  // + 8*slot
+    const uint32_t b_odone0 = b_qfull + 48;   // + 8*slot
+    const uint32_t b_oempty0 = b_qfull + 64;  // + 8*slot
+    const uint32_t b_drain = b_qfull + 80;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::BAR_OFF + 16u * NST + 96);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + 16u * NST + 100);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NST; ++i) {
+            mbar_init(full_bar(i), 1);
+            mbar_init(empty_bar(i), 1);
+        }
+        mbar_init(b_qfull, 1);
+        mbar_init(b_qempty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(b_sfull0 + 8 * s, 1);
+            mbar_init(b_pready0 + 8 * s, 128);
+            mbar_init(b_odone0 + 8 * s, 1);
+            mbar_init(b_oempty0 + 8 * s, 128);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tm_q);
+        prefetch_tmap(&p.tm_k);
+        prefetch_tmap(&p.tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32((const void*)tmem_slot), 512);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int n_items = (p.mode == 0) ? p.n_items : *p.n_items_dev;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------------------ producer
+        int kv_it = 0, q_it = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+            PrefillItem it;
+            prefill_get_item(p, idx, it);
+            if (it.n_kv == 0) continue;
+            if (!mbar_wait(b_qempty, (q_it & 1) ^ 1, abort_flag)) { ok = false; break; }
+            mbar_arrive_expect_tx(b_qfull, it.nh * TILE);
+            for (int s = 0; s < it.nh; ++s)
+                for (int hf = 0; hf < C::HALVES; ++hf)
+                    tma_load_4d(sQ + s * TILE + hf * 16384u, &p.tm_q, b_qfull, hf * 64, it.h0 + s,
+                                it.q_tok0, it.batch);
+            ++q_it;
+            const int g = it.h0 / p.G;
+            for (int j = 0; ok && j < it.n_kv; ++j) {
+                for (int t = 0; t < 2; ++t) {
+                    const int st = kv_it % NST;
+                    if (!mbar_wait(empty_bar(st), ((kv_it / NST) & 1) ^ 1, abort_flag)) { ok = false; break; }
+                    mbar_arrive_expect_tx(full_bar(st), TILE);
+                    const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
+                    for (int hf = 0; hf < C::HALVES; ++hf)
+                        tma_load_4d(sKV + st * TILE + hf * 16384u, map, full_bar(st), hf * 64, g,
+                                    it.kv_tok0 + j * 128, it.batch);
+                    ++kv_it;
+                }
+            }
+        }
+        // Let every load this thread issued land before the block exits.
+        const int n_last = min(kv_it, NST);
+        for (int k = kv_it - n_last; k < kv_it; ++k)
+            mbar_wait(full_bar(k % NST), (k / NST) & 1, nullptr, 100000000ull);
+        if (q_it > 0) mbar_wait(b_qfull, (q_it - 1) & 1, nullptr, 100000000ull);
+    } else if (warp == 1 && lane == 0) {
+        // --------------------------------------------------------- MMA issuer
+        int kv_it = 0, q_it = 0;
+        int pr_cnt[2] = {0, 0}, oe_cnt[2] = {0, 0};
+        bool ok = true;
+        auto issue_qk = [&](int s, int st) {
+            const uint32_t d_tmem = tmem + 128u * s;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+                const uint64_t a = smem_desc_sw128(sQ + s * TILE + off, 16, 1024);
+                const uint64_t b = smem_desc_sw128(sKV + st * TILE + off, 16, 1024);
+                tc_mma_ss(d_tmem, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+        };
+        auto issue_pv = [&](int s, int st, bool acc) {
+            const uint32_t d_tmem = tmem + 256u + (uint32_t)(D * s);
+            const uint32_t a_tmem = tmem + 128u * s;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t b = smem_desc_sw128(sKV + st * TILE + kk * 2048u, 16384, 1024);
+                tc_mma_ts(d_tmem, a_tmem + kk * 8u, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+            }
+        };
+        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+            PrefillItem it;
+            prefill_get_item(p, idx, it);
+            if (it.n_kv == 0) continue;
+            if (!mbar_wait(b_qfull, q_it & 1, abort_flag)) { ok = false; break; }
+            ++q_it;
+            // prologue: S = Q K(0)^T for both slots
+            int stK = kv_it % NST;
+            if (!mbar_wait(full_bar(stK), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
+            ++kv_it;
+            tc_fence_after();
+            for (int s = 0; s < it.nh; ++s) {
+                issue_qk(s, stK);
+                tc_commit(b_sfull0 + 8 * s);
+            }
+            tc_commit(empty_bar(stK));
+            if (it.n_kv == 1) tc_commit(b_qempty);
+            for (int j = 0; ok && j < it.n_kv; ++j) {
+                const int stV = kv_it % NST;
+                if (!mbar_wait(full_bar(stV), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
+                ++kv_it;
+                const bool more = (j + 1 < it.n_kv);
+                const int stK1 = kv_it % NST;
+                const uint32_t parK1 = (kv_it / NST) & 1;
+                for (int s = 0; ok && s < it.nh; ++s) {
+                    if (!mbar_wait(b_pready0 + 8 * s, pr_cnt[s] & 1, abort_flag)) { ok = false; break; }
+                    ++pr_cnt[s];
+                    if (j == 0) {
+                        if (!mbar_wait(b_oempty0 + 8 * s, (oe_cnt[s] & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        ++oe_cnt[s];
+                    }
+                    tc_fence_after();
+                    issue_pv(s, stV, j > 0);
+                    tc_commit(b_odone0 + 8 * s);
+                    if (more) {
+                        if (s == 0) {
+                            if (!mbar_wait(full_bar(stK1), parK1, abort_flag)) { ok = false; break; }
+                            tc_fence_after();
+                        }
+                        issue_qk(s, stK1);
+                        tc_commit(b_sfull0 + 8 * s);
+                    }
+                }
+                if (!ok) break;
+                tc_commit(empty_bar(stV));
+                if (more) {
+                    ++kv_it;
+                    tc_commit(empty_bar(stK1));
+                    if (j + 2 == it.n_kv) tc_commit(b_qempty);
+                }
+            }
+        }
+        // Wait for every MMA this thread issued before TMEM is released.
+        tc_commit(b_drain);
+        mbar_wait(b_drain, 0, nullptr, 100000000ull);
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax
+        const int slot = (warp - 4) >> 2;
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t tS = tmem + lane_off + 128u * slot;
+        const uint32_t tO = tmem + lane_off + 256u + (uint32_t)(D * slot);
+        const uint32_t b_sfull = b_sfull0 + 8 * slot, b_pready = b_pready0 + 8 * slot;
+        const uint32_t b_odone = b_odone0 + 8 * slot, b_oempty = b_oempty0 + 8 * slot;
+        const float sl2 = p.scale_log2;
+        int sf_cnt = 0, od_base = 0;
+        bool ok = true;
+        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+            PrefillItem it;
+            prefill_get_item(p, idx, it);
+            if (slot >= it.nh) continue;
+            const int h = it.h0 + slot;
+            const int row = it.qt * 128 + r;
+            const bool valid = row < it.Lq;
+            const int tok = it.q_tok0 + r;
+            __nv_bfloat16* orow = p.o + (int64_t)it.batch * p.o_bs + (int64_t)tok * p.o_ts + (int64_t)h * p.o_hs;
+            float m_use = -INFINITY, l = 0.f;
+            if (it.n_kv > 0) {
+                const int lim = p.causal ? min(it.Lkv, row + it.Lkv - it.Lq + 1) : it.Lkv;
+                for (int j = 0; j < it.n_kv; ++j) {
+                    if (!mbar_wait(b_sfull, sf_cnt & 1, abort_flag)) { ok = false; break; }
+                    ++sf_cnt;
+                    tc_fence_after();
+                    float x[128];
+                    {
+                        uint32_t u[32];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            tmem_ld32(tS + 32u * c, u);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(u[e]);
+                        }
+                    }
+                    const int kb = j * 128;
+                    float mx = -INFINITY;
+                    if (kb + 128 > lim) {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c) {
+                            x[c] = (kb + c < lim) ? x[c] * sl2 : -INFINITY;
+                            mx = fmaxf(mx, x[c]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 128; ++c) {
+                            x[c] *= sl2;
+                            mx = fmaxf(mx, x[c]);
+                        }
+                    }
+                    const float m_new = fmaxf(m_use, mx);
+                    float alpha = 1.f;
+                    const bool old_finite = (m_use != -INFINITY);
+                    if (m_new > m_use + 8.f) {
+                        alpha = ex2(m_use - m_new);
+                        m_use = m_new;
+                    }
+                    const float mref = (m_use == -INFINITY) ? 0.f : m_use;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const float p0 = ex2(x[32 * c + 2 * e] - mref);
+                            const float p1 = ex2(x[32 * c + 2 * e + 1] - mref);
+                            sum += p0 + p1;
+                            pk[e] = pack_bf16(p0, p1);
+                        }
+                        tmem_st16(tS + 16u * c, pk);
+                    }
+                    l = l * alpha + sum;
+                    const bool need_o = (j > 0) && old_finite && (alpha != 1.f);
+                    if (__any_sync(0xffffffffu, need_o)) {
+                        // PV(j-1) must have landed in O before it is rescaled.
+                        if (!mbar_wait(b_odone, (od_base + j - 1) & 1, abort_flag)) { ok = false; }
+                        tc_fence_after();
+                        const float f = need_o ? alpha : 1.f;
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t u[32];
+                            tmem_ld32(tO + 32u * c, u);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
+                            tmem_st32(tO + 32u * c, u);
+                        }
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(b_pready);
+                    if (!ok) break;
+                }
+                if (!ok) break;
+                // epilogue: O / l -> bf16
+                if (!mbar_wait(b_odone, (od_base + it.n_kv - 1) & 1, abort_flag)) { ok = false; break; }
+                od_base += it.n_kv;
+                tc_fence_after();
+                const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tO + 32u * c, u);
+                    tc_wait_ld();
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(u[8 * v4 + 0]) * inv_l, __uint_as_float(u[8 * v4 + 1]) * inv_l);
+                            w.y = pack_bf16(__uint_as_float(u[8 * v4 + 2]) * inv_l, __uint_as_float(u[8 * v4 + 3]) * inv_l);
+                            w.z = pack_bf16(__uint_as_float(u[8 * v4 + 4]) * inv_l, __uint_as_float(u[8 * v4 + 5]) * inv_l);
+                            w.w = pack_bf16(__uint_as_float(u[8 * v4 + 6]) * inv_l, __uint_as_float(u[8 * v4 + 7]) * inv_l);
+                            dst[v4] = w;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(b_oempty);
+            } else if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow);
+                for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
+            }
+            if (valid && p.lse != nullptr) {
+                const float lse = (l > 0.f) ? (m_use + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                int64_t li;
+                if (p.lse_layout == 0) li = ((int64_t)it.b * p.Hq + h) * p.Sq + row;
+                else if (p.lse_layout == 1) li = ((int64_t)it.b * p.lse_smax + row) * p.Hq + h;
+                else li = (int64_t)tok * p.Hq + h;
+                p.lse[li] = lse;
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace b2

@@ -1,0 +1,137 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/b2attn.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ragged_scaled_dot_b200 as rsd
+from ragged_scaled_dot_b200 import build as rsd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "b2attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rsd_build.build()
+    return rsd.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("attn_fwd_dense", "attn_fwd_ragged", "attn_fwd_paged", "attn_split_merge"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in rsd.SIGNATURES, f"binding lacks {n}"
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert rsd.status_string(code).startswith("ATTN_")
+    assert rsd.status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    # ragged: header + one 16-byte item per (query tile, head group)
+    n = rsd.attn_fwd_ragged_workspace_size(2, 64, 101, 4, 1)
+    assert n == 256 + min(101 // 128 + 2, 2 * 1) * 2 * 16
+    assert rsd.attn_fwd_ragged_workspace_size(0, 64, 101, 4, 1) == 0
+    # paged: none for one split; partial O (fp32) + partial LSE otherwise
+    assert rsd.attn_fwd_paged_workspace_size(128, 64, 128, 1) == 0
+    n = rsd.attn_fwd_paged_workspace_size(128, 64, 128, 3)
+    assert n >= 3 * 128 * 64 * 128 * 4 + 3 * 128 * 64 * 4 and n % 256 == 0
+
+
+def test_suggest_splits_range(lib):
+    for args in [(128, 64, 8, 128, 128, 32768, 64, 148), (64, 128, 1, 576, 512, 65536, 64, 148),
+                 (1, 8, 1, 128, 128, 64, 16, 148), (4096, 32, 8, 128, 128, 1024, 64, 148)]:
+        s = rsd.attn_paged_suggest_splits(*args)
+        assert 1 <= s <= 64
+
+
+L2 = ctypes.c_int64 * 2
+L3 = ctypes.c_int64 * 3
+
+
+def test_dense_rejects_bad_args_on_host(lib):
+    st = L3(8 * 4 * 64, 4 * 64, 64)
+    f = lib.attn_fwd_dense
+    # Hq not a multiple of Hkv
+    assert f(None, None, None, None, None, 1, 8, 8, 3, 2, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_INVALID_ARG
+    # unsupported head dim
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 96, 96, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_UNSUPPORTED
+    # non-finite scale
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, float("nan"), 1, None) == rsd.ATTN_ERR_INVALID_ARG
+    # empty problem is a no-op
+    assert f(None, None, None, None, None, 0, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_OK
+    # null pointers with a real shape
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_INVALID_ARG
+
+
+def test_ragged_requires_workspace(lib):
+    s2 = L2(4 * 64, 64)
+    f = lib.attn_fwd_ragged
+    fake = ctypes.c_void_p(0x100000)  # never dereferenced: rejected before launch
+    rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
+           s2, s2, s2, s2, 0, 0.125, 1, None, 0, None)
+    assert rc == rsd.ATTN_ERR_WORKSPACE
+    rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
+           s2, s2, s2, s2, 0, 0.125, 1, ctypes.c_void_p(0x100100), 8, None)
+    assert rc == rsd.ATTN_ERR_WORKSPACE
+    # bad LSE layout code
+    rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
+           s2, s2, s2, s2, 7, 0.125, 1, None, 0, None)
+    assert rc == rsd.ATTN_ERR_INVALID_ARG
+
+
+def test_paged_rejects_bad_args_on_host(lib):
+    f = lib.attn_fwd_paged
+    fake = ctypes.c_void_p(0x100000)
+    q2 = L2(64 * 128, 128)
+    kp = L3(8 * 64 * 128, 128, 64 * 128)
+    args = dict(B=4, Hq=64, Hkv=8, Dqk=128, Dv=128, ps=64, P=100, maxkv=4096, splits=3)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(fake, fake, fake, fake, None, fake, 64, fake, a["B"], a["Hq"], a["Hkv"], a["Dqk"],
+                 a["Dv"], a["ps"], a["P"], a["maxkv"], q2, q2, kp, kp, 0.088, a["splits"], None, 0,
+                 None)
+
+    assert call() == rsd.ATTN_ERR_WORKSPACE              # 3 splits need a workspace
+    assert call(Dqk=96, Dv=96) == rsd.ATTN_ERR_UNSUPPORTED
+    assert call(ps=48) == rsd.ATTN_ERR_UNSUPPORTED        # neither divides nor is divided by 64
+    assert call(Hkv=7) == rsd.ATTN_ERR_INVALID_ARG        # 64 % 7 != 0
+    assert call(Hq=256, Hkv=8) == rsd.ATTN_ERR_UNSUPPORTED  # G = 32 > 16
+    assert call(Dqk=576, Dv=512, Hq=128, Hkv=2) == rsd.ATTN_ERR_UNSUPPORTED  # MLA needs one KV head
+    assert call(splits=0) == rsd.ATTN_ERR_INVALID_ARG
+
+
+def test_merge_rejects_bad_args_on_host(lib):
+    f = lib.attn_split_merge
+    fake = ctypes.c_void_p(0x100000)
+    assert f(fake, fake, 0, 10, 128, fake, 128, None, None) == rsd.ATTN_ERR_INVALID_ARG
+    assert f(fake, fake, 2, 10, 96, fake, 96, None, None) == rsd.ATTN_ERR_UNSUPPORTED
+    assert f(fake, fake, 2, 10, 128, fake, 64, None, None) == rsd.ATTN_ERR_INVALID_ARG
+    assert f(None, None, 2, 0, 128, None, 128, None, None) == rsd.ATTN_OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(rsd, "_lib", None)
+    monkeypatch.setattr(rsd, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        rsd.lib()

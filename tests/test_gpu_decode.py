@@ -1,0 +1,136 @@
+"""Paged decode (GQA and absorbed MLA) with split-KV on the GPU vs the fp64
+oracle, plus paged == contiguous (bit-exact), split == unsplit, NaN in the
+unused tail of the last page, and the standalone LSE merge."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ragged_scaled_dot_b200 as rsd
+import synth
+from gpu_util import assert_lse_close, assert_o_close, bits, check_paged, orc, paged_gpu
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _paged_inputs(lens, Hq, Hkv, D, ps, seed, layout="HND", Dv=None, alias=False, extra_pages=3):
+    table, total = synth.page_table(lens, ps, seed)
+    P = total + extra_pages
+    q = synth.normal_bf16((len(lens), Hq, D), seed + 1, "cpu").to(DEV)
+    shape_k = (P, Hkv, ps, D) if layout == "HND" else (P, ps, Hkv, D)
+    k = synth.normal_bf16(shape_k, seed + 2, "cpu").to(DEV)
+    if alias:
+        v = k
+    else:
+        Dv = Dv or D
+        shape_v = (P, Hkv, ps, Dv) if layout == "HND" else (P, ps, Hkv, Dv)
+        v = synth.normal_bf16(shape_v, seed + 3, "cpu").to(DEV)
+    return q, k, v, table, np.asarray(lens, dtype=np.int32)
+
+
+GQA_CASES = [
+    # (lens, Hq, Hkv, D, ps, layout, splits)
+    ([0, 1, 63, 64, 1000], 16, 2, 128, 64, "HND", 1),
+    ([0, 1, 63, 64, 1000], 16, 2, 128, 64, "HND", 3),
+    ([65, 700, 2049], 64, 8, 128, 64, "HND", 7),
+    ([5, 300, 129], 8, 1, 128, 16, "NHD", 2),
+    ([100, 1, 777], 32, 4, 64, 32, "HND", 4),
+    ([1000, 20], 4, 4, 128, 128, "NHD", 2),
+    ([3000], 12, 1, 128, 64, "HND", 16),   # more splits than some sequences have pages
+]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,ps,layout,splits", GQA_CASES)
+def test_gqa_decode_cases(lens, Hq, Hkv, D, ps, layout, splits):
+    q, k, v, table, kl = _paged_inputs(lens, Hq, Hkv, D, ps, seed=len(lens) * 11 + ps, layout=layout)
+    check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(D), splits, kv_layout=layout,
+                where=f"gqa {lens} ps{ps} S{splits}")
+
+
+def test_paged_equals_contiguous_bitwise():
+    """A random page permutation gives bit-identical results to the identity
+    table over a pool pre-permuted so both see the same logical K/V."""
+    lens = [500, 64, 1100]
+    Hq, Hkv, D, ps = 16, 2, 128, 64
+    q, k, v, table, kl = _paged_inputs(lens, Hq, Hkv, D, ps, seed=3)
+    o1, l1 = paged_gpu(q, k, v, table, kl, ps, 0.09, 1)
+    # identity layout: logical page i of the batch stored at physical i
+    n_pages = [(L + ps - 1) // ps for L in lens]
+    phys = np.concatenate([table[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
+    k2 = k[torch.as_tensor(phys, device=DEV)].contiguous()
+    v2 = v[torch.as_tensor(phys, device=DEV)].contiguous()
+    t2 = np.full_like(table, -1)
+    pos = 0
+    for b, n in enumerate(n_pages):
+        t2[b, :n] = np.arange(pos, pos + n)
+        pos += n
+    o2, l2 = paged_gpu(q, k2, v2, t2, kl, ps, 0.09, 1)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_split_equals_unsplit():
+    lens = [4000, 129, 64, 1]
+    q, k, v, table, kl = _paged_inputs(lens, 16, 2, 128, 64, seed=7)
+    o1, l1 = paged_gpu(q, k, v, table, kl, 64, 0.09, 1)
+    for S in (2, 7, 63):
+        o2, l2 = paged_gpu(q, k, v, table, kl, 64, 0.09, S)
+        assert_o_close(o2, o1.float().cpu().numpy().astype(np.float64), f"split {S}")
+        assert np.max(np.abs(l2.cpu().numpy() - l1.cpu().numpy())) < 1e-4
+
+
+def test_nan_inside_last_page_is_never_used():
+    """Slots past kv_len inside a sequence's last page hold NaN: outputs stay
+    finite and equal to a run with clean slots."""
+    lens = [70, 200]
+    ps = 64
+    q, k, v, table, kl = _paged_inputs(lens, 8, 1, 128, ps, seed=17)
+    kn, vn = k.clone(), v.clone()
+    for b, L in enumerate(lens):
+        last = table[b, (L - 1) // ps]
+        kn[last, :, L % ps:] = float("nan")
+        vn[last, :, L % ps:] = float("nan")
+    for S in (1, 3):
+        o1, l1 = paged_gpu(q, k, v, table, kl, ps, 0.1, S)
+        o2, l2 = paged_gpu(q, kn, vn, table, kl, ps, 0.1, S)
+        assert torch.isfinite(o2.float()).all()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+@pytest.mark.parametrize("alias", [True, False])
+def test_mla_decode(splits, alias):
+    lens = [0, 100, 700, 33]
+    Hq, D, Dv, ps = 128, 576, 512, 64
+    q, k, v, table, kl = _paged_inputs(lens, Hq, 1, D, ps, seed=23, Dv=Dv, alias=alias)
+    check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(D), splits, Dv=Dv,
+                where=f"mla alias={alias} S={splits}")
+
+
+def test_mla_nan_past_kv_len_aliased():
+    lens = [90]
+    ps = 64
+    q, k, _, table, kl = _paged_inputs(lens, 128, 1, 576, ps, seed=29, alias=True)
+    kn = k.clone()
+    kn[table[0, 1], :, 90 - 64:] = float("nan")
+    o1, l1 = paged_gpu(q, k, k, table, kl, ps, 0.04, 1, o_dv=512)
+    o2, l2 = paged_gpu(q, kn, kn, table, kl, ps, 0.04, 1, o_dv=512)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("Dv", [64, 128, 512])
+def test_split_merge_kernel_vs_oracle(Dv):
+    S, R = 5, 300
+    g = torch.Generator().manual_seed(Dv)
+    o_part = torch.randn((S, R, Dv), generator=g)
+    lse_part = torch.randn((S, R), generator=g) * 3
+    lse_part[torch.rand((S, R), generator=g) < 0.3] = -float("inf")
+    lse_part[:, :7] = -float("inf")              # rows with no keys at all
+    o_part[lse_part == -float("inf")] = float("nan")  # empty partials must be ignored
+    o_ref, l_ref = orc().split_merge(o_part.numpy(), lse_part.numpy())
+    o = torch.full((R, Dv), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((R,), dtype=torch.float32, device=DEV)
+    rsd.attn_split_merge(o_part.to(DEV), lse_part.to(DEV), o, lse)
+    torch.cuda.synchronize()
+    assert_o_close(o, o_ref, "merge")
+    assert_lse_close(lse, l_ref, "merge")
