@@ -140,8 +140,12 @@ class Part:
         self.info = info or {}
 
 
-def make_ragged_prefill(torch, rsd, synth, dev, seed_offset):
-    w = synth.WORKLOADS["ragged_prefill"]
+def _with_batch(synth, w, B):
+    return w if not B else synth.Workload(**{**w.__dict__, "B": B})
+
+
+def make_ragged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
+    w = _with_batch(synth, synth.WORKLOADS["ragged_prefill"], B)
     L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
     q, k, v, cu = synth.make_ragged(w, dev, lengths=L)
     T = q.shape[0]
@@ -184,8 +188,8 @@ def make_ragged_prefill(torch, rsd, synth, dev, seed_offset):
     return Part("ragged_prefill", "TFLOP/s", flops / 1e12, 3, step, e2e_setup, info), data
 
 
-def make_dense_prefill(torch, rsd, synth, dev, seed_offset):
-    w = synth.WORKLOADS["dense_prefill"]
+def make_dense_prefill(torch, rsd, synth, dev, seed_offset, B=0):
+    w = _with_batch(synth, synth.WORKLOADS["dense_prefill"], B)
     g = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
     q, k, v = synth.make_dense(g, dev)
     o = torch.empty_like(q)
@@ -198,8 +202,8 @@ def make_dense_prefill(torch, rsd, synth, dev, seed_offset):
     return Part("dense_prefill", "TFLOP/s", flops / 1e12, 1, step, None, info), None
 
 
-def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms):
-    w = synth.WORKLOADS[name]
+def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
+    w = _with_batch(synth, synth.WORKLOADS[name], B)
     L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
     q, kp, vp, table, kl = synth.make_paged(w, dev, kv_lens=L)
     Dv = w.Dv
@@ -431,7 +435,7 @@ def run_ours(args):
     d_val, d_ms, d_roof = part_summary(decode, "hbm")
 
     e2e = {}
-    for part in (prefill, decode):
+    for part in ((prefill, decode) if not args.no_e2e else ()):
         ms, h2d, d2h = time_e2e(torch, part, max(1, min(3, args.steps)), dist)
         e2e[part.name] = {"value": round(part.units * world / (ms / 1e3 / max(1, min(3, args.steps))), 3),
                           "unit": part.unit, "h2d_bytes_per_step": int(h2d),
@@ -480,9 +484,9 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (126 MB); no flush needed",
                        "prefill": prefill.info, "decode": decode.info},
             "roofline": p_roof,
-            "e2e": e2e["ragged_prefill"],
+            "e2e": e2e.get("ragged_prefill"),
             "decode": {"metric": "paged-decode KV GB/s", "value": round(d_val, 1), "unit": "GB/s",
-                       "ms_per_step": round(d_ms, 4), "roofline": d_roof, "e2e": e2e["paged_decode"]},
+                       "ms_per_step": round(d_ms, 4), "roofline": d_roof, "e2e": e2e.get("paged_decode")},
             "extras": extra_out,
             "gpu_launches": args.steps * (prefill.launches + decode.launches)
                             + sum(args.steps * p.launches for p in extras),
@@ -495,6 +499,28 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_one(args):
+    """Profiling helper: build one part (optionally with a smaller batch), run
+    warm-up + timed steps, print a short JSON line.  Not the benchmark line."""
+    import torch
+    import ragged_scaled_dot_b200 as rsd
+    import synth
+    torch.cuda.set_device(0)
+    rsd.lib()
+    num_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if args.only == "ragged_prefill":
+        part = make_ragged_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
+    elif args.only == "dense_prefill":
+        part = make_dense_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
+    else:
+        part = make_paged(torch, rsd, synth, "cuda", 0, args.only, num_sms, args.batch)[0]
+    total_ms, per = time_part(torch, part, args.steps, args.warmup, None, 1)
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    print(json.dumps({"part": part.name, "unit": part.unit, "units_per_step": part.units,
+                      "ms_per_step": total_ms / args.steps,
+                      "value": part.units / (total_ms / 1e3 / args.steps), "info": part.info}), flush=True)
 
 
 # --------------------------------------------------------------------------- #
@@ -545,11 +571,17 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "mla_decode"],
+                    help="profiling: time one part only and print its own line")
+    ap.add_argument("--batch", type=int, default=0, help="profiling: override the part's batch size")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        run_one(args)
     else:
         run_ours(args)
 
