@@ -134,6 +134,38 @@ size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q,
                                       int Hq, int Hkv);
 
 /*
+ * attn_fwd_ragged without a workspace argument, for callers that cannot
+ * allocate device memory when they call (the release pages have no
+ * counterpart; this entry point is specific to this library).  Typical
+ * callers: code that runs inside a CUDA stream capture, where a cudaMalloc
+ * would invalidate the capture, and plugins or runtimes whose host framework
+ * owns all device memory and forbids allocation during execution.
+ * The work list lives in a 4 MiB array built into the library instead
+ * (attn_fwd_ragged_noalloc_max_scratch() returns the size); every GPU that
+ * loads the library holds it until the process exits.  Arguments, layouts
+ * and results are those of attn_fwd_ragged.
+ *  - Capacities whose work list needs more than 4 MiB
+ *    (attn_fwd_ragged_workspace_size(...) > 4 MiB) return ATTN_ERR_WORKSPACE.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - All calls share the one array, and each call rewrites it before use.
+ *    Calls that overlap on the GPU (e.g. issued on two streams without an
+ *    ordering between them) race on it: order them on one stream.
+ *  - It allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+int attn_fwd_ragged_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_kv,
+                            int B, int max_seqlen_q, int max_seqlen_kv,
+                            int64_t total_q, int64_t total_kv,
+                            int Hq, int Hkv, int Dqk, int Dv,
+                            const int64_t q_strides[2], const int64_t k_strides[2],
+                            const int64_t v_strides[2], const int64_t o_strides[2],
+                            int lse_layout, float scale, int causal, void *stream);
+
+/* Bytes of the built-in scratch attn_fwd_ragged_noalloc uses (4 MiB). */
+size_t attn_fwd_ragged_noalloc_max_scratch(void);
+
+/*
  * Paged-KV decode forward: one query token per sequence, attending to all of
  * its kv_lens[b] cached keys ("cuDNN Frontend v1.31.0 Release Notes", "SDPA:
  * paged KV, split-KV, and engine selection").

@@ -39,6 +39,9 @@ SIGNATURES = {
     "attn_fwd_ragged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _L, _I, _I, _I, _I,
                              _L2, _L2, _L2, _L2, _I, _F, _I, _P, _Z, _P]),
     "attn_fwd_ragged_workspace_size": (_Z, [_I, _I, _L, _I, _I]),
+    "attn_fwd_ragged_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _L, _I, _I, _I, _I,
+                                     _L2, _L2, _L2, _L2, _I, _F, _I, _P]),
+    "attn_fwd_ragged_noalloc_max_scratch": (_Z, []),
     "attn_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _I, _I, _I, _I, _L, _I,
                             _L2, _L2, _L3, _L3, _F, _I, _P, _Z, _P]),
     "attn_fwd_paged_workspace_size": (_Z, [_I, _I, _I, _I]),
@@ -141,6 +144,34 @@ def attn_fwd_ragged(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_
         B, int(max_seqlen_q), int(max_seqlen_kv), int(total_q), int(total_kv), Hq, Hkv, Dqk, Dv,
         st(q), st(k), st(v), st(o), int(lse_layout), float(scale), int(causal),
         _ptr(workspace), ws_bytes, _stream(stream)), "attn_fwd_ragged")
+
+
+def attn_fwd_ragged_noalloc(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_kv, *, max_seqlen_q: int,
+                            max_seqlen_kv: int, scale: float, causal: bool,
+                            lse_layout: int = ATTN_LSE_PADDED_BSH, total_q=None, total_kv=None,
+                            stream=None):
+    """attn_fwd_ragged for callers that cannot allocate device memory at call
+    time (inside a stream capture, or under a framework that owns all device
+    memory): the work list goes to a 4 MiB scratch array built into the
+    library.  Calls share that array, so calls that overlap on the GPU race;
+    the first call on a device should come before any stream capture."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bf16(t, n)
+    B = cu_seqlens_q.numel() - 1
+    Hq, Dqk = q.shape[1], q.shape[2]
+    Hkv, Dv = k.shape[1], v.shape[2]
+    total_q = q.shape[0] if total_q is None else total_q
+    total_kv = k.shape[0] if total_kv is None else total_kv
+    st = lambda t: _L2(t.stride(0), t.stride(1))  # noqa: E731
+    _check(lib().attn_fwd_ragged_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_kv),
+        B, int(max_seqlen_q), int(max_seqlen_kv), int(total_q), int(total_kv), Hq, Hkv, Dqk, Dv,
+        st(q), st(k), st(v), st(o), int(lse_layout), float(scale), int(causal), _stream(stream)),
+        "attn_fwd_ragged_noalloc")
+
+
+def attn_fwd_ragged_noalloc_max_scratch() -> int:
+    return int(lib().attn_fwd_ragged_noalloc_max_scratch())
 
 
 # --------------------------------------------------------------------- paged

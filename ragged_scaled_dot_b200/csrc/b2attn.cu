@@ -126,6 +126,32 @@ void pair_shape(int Hq, int Hkv, int* hpi, int* n_pairs) {
     *n_pairs = Hq / *hpi;
 }
 
+// ---------------------------------------------------------------------------
+// Built-in scratch for attn_fwd_ragged_noalloc: holds the ragged work list for
+// callers that may not allocate device memory.  Every GPU that loads this
+// library keeps these bytes reserved until the process exits.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device.  In host code the symbol is only a host-side stand-in, so the
+// kernel must be given the address cudaGetSymbolAddress returns.
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ATTN_OK;
+}
+
 // Launches the prefill kernel for an already-filled PrefillParams.
 int launch_prefill(PrefillParams& pp, int D, int grid, cudaStream_t st) {
     if (grid <= 0) return ATTN_OK;
@@ -303,6 +329,24 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     const int grid = (int)(items_max < sms ? items_max : sms);
     return launch_prefill(pp, D, grid, st);
 }
+
+// --------------------------------------------------- ragged, no allocation
+int attn_fwd_ragged_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_kv, int B, int max_seqlen_q,
+                            int max_seqlen_kv, int64_t total_q, int64_t total_kv, int Hq, int Hkv, int Dqk,
+                            int Dv, const int64_t q_strides[2], const int64_t k_strides[2],
+                            const int64_t v_strides[2], const int64_t o_strides[2], int lse_layout, float scale,
+                            int causal, void* stream) {
+    const size_t need = attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
+    if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;  // work list would not fit 4 MiB
+    void* scratch = nullptr;
+    if (int e = noalloc_scratch(&scratch)) return e;
+    return attn_fwd_ragged(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv, total_q,
+                           total_kv, Hq, Hkv, Dqk, Dv, q_strides, k_strides, v_strides, o_strides, lse_layout,
+                           scale, causal, scratch, kNoAllocScratchBytes, stream);
+}
+
+size_t attn_fwd_ragged_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
 
 // ------------------------------------------------------------------ paged
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits) {
