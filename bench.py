@@ -37,6 +37,12 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill attention TFLOPS and paged-decode KV GB/s, % of B200 roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# DRAM bytes (read + write) per algorithmic unit from the latest ncu capture of
+# each kernel (profiles/), scaled to a full launch by units processed.  None
+# when the kernel changed after the counters were taken.
+#   paged_decode: profiles/decode_gqa_kernel_paged_b32.md (2.692 GB / 2.673 GB)
+TRAFFIC_PER_UNIT = {"ragged_prefill": None, "paged_decode": 1.0071}
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -419,15 +425,21 @@ def run_ours(args):
         if bound == "tensor":
             achieved = part.units / (kern_ms / 1e3)
             peak = peaks["bf16_tflops"]
+            tpu = TRAFFIC_PER_UNIT.get(part.name)
             roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "frac": round(achieved / peak, 4),
+                    "traffic": None if tpu is None else round(part.units * tpu, 3),
+                    "traffic_unit": "GB per launch (dram read + write)",
                     "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
                     "peak_source": f"{peak_src} bf16_tflops (burst)"}
         else:
             achieved = part.units / (kern_ms / 1e3)
             peak = peaks["hbm_gbs"]
+            tpu = TRAFFIC_PER_UNIT.get(part.name)
             roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "frac": round(achieved / peak, 4),
+                    "traffic": None if tpu is None else round(part.units * tpu, 3),
+                    "traffic_unit": "GB per launch (dram read + write)",
                     "peak_source": f"{peak_src} hbm_gbs"}
         return value, ms, roof
 

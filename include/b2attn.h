@@ -241,6 +241,16 @@ int attn_get_device_error(void *stream);
  */
 int attn_selftest_bounded_wait(uint64_t timeout_ns, void *stream);
 
+/*
+ * Diagnostic: y[i] = 2^t[i] evaluated the way the prefill softmax evaluates
+ * the share of its exponentials it moves off the MUFU unit onto the FMA pipe
+ * (base-2 range reduction n = round(t), f = t - n, a degree-3 polynomial for
+ * 2^f, n added to the exponent; "cuDNN Frontend v1.30.0 Release Notes", "SDPA:
+ * more kernels and numerics": exp2 on the FMA pipe).  Inputs below -125 give
+ * 2^-125.  t and y are device arrays of n floats.
+ */
+int attn_selftest_exp2(const float *t, float *y, int64_t n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -49,6 +49,7 @@ SIGNATURES = {
     "attn_split_merge": (_I, [_P, _P, _I, _L, _I, _P, _L, _P, _P]),
     "attn_get_device_error": (_I, [_P]),
     "attn_selftest_bounded_wait": (_I, [_U64, _P]),
+    "attn_selftest_exp2": (_I, [_P, _P, _L, _P]),
 }
 
 _lib = None
@@ -232,3 +233,9 @@ def attn_get_device_error(stream=None) -> int:
 def attn_selftest_bounded_wait(timeout_ns: int, stream=None):
     _check(lib().attn_selftest_bounded_wait(int(timeout_ns), _stream(stream)),
            "attn_selftest_bounded_wait")
+
+
+def attn_selftest_exp2(t, y, stream=None):
+    """y = 2**t through the prefill softmax's FMA-pipe exponential (fp32 CUDA tensors)."""
+    _check(lib().attn_selftest_exp2(_ptr(t), _ptr(y), int(t.numel()), _stream(stream)),
+           "attn_selftest_exp2")

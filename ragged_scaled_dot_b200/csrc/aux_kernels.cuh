@@ -9,13 +9,18 @@ namespace b2 {
 // ---------------------------------------------------------------------------
 // Ragged work list, built on the device from the offset tables so the host
 // never reads them back ("cuDNN Frontend v1.28.0 release notes", "Ragged /
-// THD, with zero host reads").  One block:
+// THD, with zero host reads"; "cuDNN Frontend v1.32.0 Release Notes", native
+// THD metadata setup fused on the device, work prefixes).  One block:
 //   1. validate each sequence against the host-declared capacities;
-//   2. histogram the work items by cost (KV tiles to visit);
-//   3. counting-sort them longest first (LPT) into `items`.
-// Items of one (sequence, query tile) are adjacent, one per query-head group.
+//   2. order sequences longest first (counting sort on query-tile count);
+//   3. give each sequence a contiguous run of items, ordered
+//      (kv head, query tile longest first, head pair), so that the CTAs that
+//      take consecutive items read the same sequence-head's K/V from L2.
+// Workspace: int header[64] (header[0] = item count, header[1] = the
+// scheduler's claim counter, zeroed here), then int4 items[max_items], then
+// two int arrays of B entries (sorted tile counts and ranks).
 // ---------------------------------------------------------------------------
-constexpr int kCostBuckets = 4096;
+constexpr int kSortBuckets = 4096;
 
 __device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t* cu_kv, int b,
                                               int max_sq, int max_skv, int64_t total_q,
@@ -28,58 +33,105 @@ __device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t
 
 __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv, int B, int max_sq,
-    int max_skv, int64_t total_q, int64_t total_kv, int causal, int n_pairs, int heads_per_item,
-    int4* __restrict__ items, int* __restrict__ n_items_out, int max_tiles) {
-    __shared__ int hist[kCostBuckets];
+    int max_skv, int64_t total_q, int64_t total_kv, int causal, int Hkv, int pairs_per_group,
+    int heads_per_item, int G, int* __restrict__ header, int4* __restrict__ items,
+    int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles) {
+    __shared__ int hist[kSortBuckets];
+    __shared__ int warp_sums[32];
     __shared__ int n_tiles_sh;
-    for (int i = threadIdx.x; i < kCostBuckets; i += blockDim.x) hist[i] = 0;
-    if (threadIdx.x == 0) {
+    const int tid = threadIdx.x;
+    for (int i = tid; i < kSortBuckets; i += blockDim.x) hist[i] = 0;
+    if (tid == 0) {
         n_tiles_sh = 0;
         if (cu_q[0] != 0 || cu_kv[0] != 0) record_status(ATTN_ERR_DEVICE_INPUT);
     }
     __syncthreads();
-    // pass 1: validate + histogram of costs
-    int my_tiles = 0;
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        if (!ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv)) {
+    // 1. validate, histogram of query-tile counts
+    for (int b = tid; b < B; b += blockDim.x) {
+        int nqt = 0;
+        if (ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv))
+            nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
+        else
             record_status(ATTN_ERR_DEVICE_INPUT);
-            continue;
-        }
-        const int lq = cu_q[b + 1] - cu_q[b], lk = cu_kv[b + 1] - cu_kv[b];
-        const int nqt = (lq + 127) >> 7;
-        for (int qt = 0; qt < nqt; ++qt) {
-            const int cost = min(prefill_n_kv(qt, lq, lk, causal), kCostBuckets - 1);
-            atomicAdd(&hist[cost], 1);
-        }
-        my_tiles += nqt;
+        atomicAdd(&hist[min(nqt, kSortBuckets - 1)], 1);
+        atomicAdd(&n_tiles_sh, nqt);
     }
-    atomicAdd(&n_tiles_sh, my_tiles);
     __syncthreads();
-    // exclusive scan, highest cost first (single thread: 4096 buckets)
-    if (threadIdx.x == 0) {
+    // 2. bucket starts, largest count first (one thread: 4096 buckets)
+    if (tid == 0) {
         int run = 0;
-        for (int c = kCostBuckets - 1; c >= 0; --c) {
+        for (int c = kSortBuckets - 1; c >= 0; --c) {
             const int h = hist[c];
             hist[c] = run;
             run += h;
         }
-        const int n = min(n_tiles_sh, max_tiles);
-        if (n_tiles_sh > max_tiles) record_status(ATTN_ERR_DEVICE_INPUT);
-        *n_items_out = n * n_pairs;
     }
     __syncthreads();
-    // pass 2: scatter
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    for (int b = tid; b < B; b += blockDim.x) {
+        int nqt = 0;
+        if (ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv))
+            nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
+        const int r = atomicAdd(&hist[min(nqt, kSortBuckets - 1)], 1);
+        rank_of[b] = r;
+        sorted_nqt[r] = nqt;
+    }
+    __syncthreads();
+    // exclusive scan of sorted_nqt (in place), chunked over the block
+    const int per = (B + blockDim.x - 1) / blockDim.x;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    int local = 0;
+    for (int i = lo; i < hi; ++i) local += sorted_nqt[i];
+    // block-wide exclusive scan of `local`
+    int incl = local;
+    const int lane = tid & 31, wid = tid >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += v;
+        }
+        warp_sums[lane] = w;  // inclusive prefix over warps
+    }
+    __syncthreads();
+    int run = incl - local + (wid > 0 ? warp_sums[wid - 1] : 0);
+    for (int i = lo; i < hi; ++i) {
+        const int v = sorted_nqt[i];
+        sorted_nqt[i] = run;
+        run += v;
+    }
+    __syncthreads();
+    const int n_tiles = min(n_tiles_sh, max_tiles);
+    if (tid == 0) {
+        if (n_tiles_sh > max_tiles) record_status(ATTN_ERR_DEVICE_INPUT);
+        header[0] = n_tiles * (Hkv * pairs_per_group);
+        header[1] = 0;
+    }
+    // 3. items of each sequence: (kv head, query tile longest first, head pair)
+    const int n_pairs = Hkv * pairs_per_group;
+    for (int b = tid; b < B; b += blockDim.x) {
         if (!ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv)) continue;
         const int lq = cu_q[b + 1] - cu_q[b], lk = cu_kv[b + 1] - cu_kv[b];
         const int nqt = (lq + 127) >> 7;
-        for (int qt = 0; qt < nqt; ++qt) {
-            const int cost = prefill_n_kv(qt, lq, lk, causal);
-            const int pos = atomicAdd(&hist[min(cost, kCostBuckets - 1)], 1);
-            if (pos >= max_tiles) continue;
-            for (int pr = 0; pr < n_pairs; ++pr)
-                items[(int64_t)pos * n_pairs + pr] = make_int4(b, qt, pr * heads_per_item, cost);
-        }
+        const int tile0 = sorted_nqt[rank_of[b]];  // first tile slot of this sequence
+        if (tile0 + nqt > max_tiles) continue;
+        const int64_t base = (int64_t)tile0 * n_pairs;
+        for (int g = 0; g < Hkv; ++g)
+            for (int t = 0; t < nqt; ++t) {
+                const int qt = nqt - 1 - t;
+                const int cost = prefill_n_kv(qt, lq, lk, causal);
+                for (int pr = 0; pr < pairs_per_group; ++pr) {
+                    const int64_t idx = base + ((int64_t)g * nqt + t) * pairs_per_group + pr;
+                    items[idx] = make_int4(b, qt, g * G + pr * heads_per_item, cost);
+                }
+            }
     }
 }
 
@@ -170,6 +222,16 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
         }
     }
     if (lse != nullptr && lane == 0) lse[r] = L;
+}
+
+// FMA-pipe exp2 self-test: y[i] = exp2_poly_pair applied to t[i].
+__global__ void selftest_exp2_kernel(const float* __restrict__ t, float* __restrict__ y, int64_t n) {
+    const int64_t i = 2 * (blockIdx.x * (int64_t)blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float2 a = make_float2(t[i], (i + 1 < n) ? t[i + 1] : 0.f);
+    const float2 r = exp2_poly_pair(a);
+    y[i] = r.x;
+    if (i + 1 < n) y[i + 1] = r.y;
 }
 
 // Bounded-wait self-test: waits on a barrier that nothing signals.

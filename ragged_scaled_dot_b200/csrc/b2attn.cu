@@ -126,6 +126,22 @@ void pair_shape(int Hq, int Hkv, int* hpi, int* n_pairs) {
     *n_pairs = Hq / *hpi;
 }
 
+// Ragged workspace layout: int header[64] | int4 items[max_items] | int sorted_nqt[B] | int rank_of[B]
+struct RaggedWs {
+    int64_t items_off, sorted_off, rank_off, total;
+};
+RaggedWs ragged_ws_layout(int B, int max_sq, int64_t total_q, int Hq, int Hkv) {
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int64_t tiles = ragged_max_tiles(B, max_sq, total_q);
+    RaggedWs w;
+    w.items_off = 256;
+    w.sorted_off = round_up(w.items_off + tiles * n_pairs * 16, 256);
+    w.rank_off = round_up(w.sorted_off + (int64_t)B * 4, 256);
+    w.total = round_up(w.rank_off + (int64_t)B * 4, 256);
+    return w;
+}
+
 // ---------------------------------------------------------------------------
 // Built-in scratch for attn_fwd_ragged_noalloc: holds the ragged work list for
 // callers that may not allocate device memory.  Every GPU that loads this
@@ -220,7 +236,7 @@ int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* 
     pp.Hkv = Hkv;
     pp.G = Hq / Hkv;
     pp.heads_per_item = hpi;
-    pp.n_pairs = n_pairs;
+    pp.pairs_per_group = pp.G / hpi;
     pp.Sq = Sq;
     pp.Skv = Skv;
     pp.n_qtiles = (Sq + 127) / 128;
@@ -242,10 +258,7 @@ int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* 
 // ----------------------------------------------------------------- ragged
 size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seqlen_q < 0 || total_q < 0) return 0;
-    int hpi, n_pairs;
-    pair_shape(Hq, Hkv, &hpi, &n_pairs);
-    const int64_t tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
-    return (size_t)(256 + tiles * n_pairs * 16);
+    return (size_t)ragged_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv).total;
 }
 
 int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
@@ -291,13 +304,17 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     }
     int hpi, n_pairs;
     pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int G = Hq / Hkv;
     const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
-    int* n_items_dev = static_cast<int*>(workspace);
-    int4* items = reinterpret_cast<int4*>(static_cast<char*>(workspace) + 256);
+    const RaggedWs wl = ragged_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv);
+    char* wsb = static_cast<char*>(workspace);
+    int* header = reinterpret_cast<int*>(wsb);
+    int4* items = reinterpret_cast<int4*>(wsb + wl.items_off);
 
-    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv,
-                                                   total_q, total_kv, causal, n_pairs, hpi, items, n_items_dev,
-                                                   max_tiles);
+    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
+        cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv, total_q, total_kv, causal, Hkv, G / hpi,
+        hpi, G, header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
+        max_tiles);
     if (int e = launch_status()) return e;
     if (lse != nullptr && lse_layout == ATTN_LSE_PADDED_BSH) {
         const int64_t n = (int64_t)B * max_seqlen_q * Hq;
@@ -311,11 +328,11 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     pp.Hkv = Hkv;
     pp.G = Hq / Hkv;
     pp.heads_per_item = hpi;
-    pp.n_pairs = n_pairs;
+    pp.pairs_per_group = G / hpi;
     pp.cu_q = cu_seqlens_q;
     pp.cu_kv = cu_seqlens_kv;
     pp.items = items;
-    pp.n_items_dev = n_items_dev;
+    pp.header = header;
     pp.o = static_cast<__nv_bfloat16*>(o);
     pp.o_bs = 0;
     pp.o_ts = o_strides[0];
@@ -513,6 +530,15 @@ int attn_get_device_error(void* stream) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(b2::g_device_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
     return v;
+}
+
+int attn_selftest_exp2(const float* t, float* y, int64_t n, void* stream) {
+    if (n < 0 || (n > 0 && (!t || !y))) return ATTN_ERR_INVALID_ARG;
+    if (n == 0) return ATTN_OK;
+    const int64_t blocks = (n / 2 + 255) / 256 + 1;
+    if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    b2::selftest_exp2_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(t, y, n);
+    return launch_status();
 }
 
 int attn_selftest_bounded_wait(uint64_t timeout_ns, void* stream) {

@@ -1,13 +1,18 @@
 // prefill.cuh -- forward attention prefill on tcgen05 tensor cores (sm_100a).
 //
-// One persistent CTA per SM walks a longest-first work list.  A work item is
+// One persistent CTA per SM claims work items one at a time.  A work item is
 // (sequence b, query tile of 128 rows, up to two query heads of one GQA group):
 // the two heads share every K/V tile, so each K/V byte brought on chip feeds
 // two 128x128 score tiles ("cuDNN Frontend v1.30.0 Release Notes", "New:
-// decode tiles", GQA packing; the grouping here is our own).
+// decode tiles", GQA packing; the grouping here is our own).  Items are
+// ordered (sequence longest first, kv head, query tile longest first, head
+// pair), so the CTAs working at the same time share one sequence-head's K/V
+// in L2 and the long items start first.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q tiles of the item, then K(j), V(j) into a ring.
+//   warp 0      claims items, publishes them to the other roles through a
+//               small shared-memory ring, and issues the TMA loads: Q tiles of
+//               the item, then K(j), V(j) into a ring of NST stages.
 //   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit.
 //   warps 4-7   softmax for slot 0 (query head h0), one TMEM lane (row) each.
 //   warps 8-11  softmax for slot 1 (query head h0 + 1).
@@ -15,17 +20,20 @@
 // P (bf16) overwrites the first 64 columns of its S tile and feeds the PV MMA
 // straight from TMEM.
 //
-// MMA order per KV tile j (FA4-style ping-pong between the two slots):
+// MMA order per KV tile j (ping-pong between the two slots):
 //   PV0(j) QK0(j+1) PV1(j) QK1(j+1)
 // so the tensor core computes one slot's MMAs while the other slot's softmax
 // runs.  The softmax keeps the running maximum m in the log2 domain with the
 // scale folded in ("cuDNN Frontend v1.30.0 Release Notes", stats_use_log2
-// section: the prefill kernels keep the softmax in the log2 domain) and only
-// rescales O when the maximum grows by more than 8 (P stays <= 2^8).
+// section: the prefill kernels keep the softmax in the log2 domain), only
+// rescales O when the maximum grows by more than 8 (P stays <= 2^8), and
+// evaluates part of the exponentials on the FMA pipe so the MUFU unit is not
+// the only source ("cuDNN Frontend v1.30.0 Release Notes", "SDPA: more kernels
+// and numerics": exp2 on the FMA pipe).
 //
 // Masking: bottom-right causal per sequence and ragged tails are applied by
-// select (-inf), never by multiplication, so values past a sequence's end can
-// not poison a row through 0 * NaN ("cuDNN Frontend v1.28.0 release notes",
+// select, never by multiplication, so values past a sequence's end can not
+// poison a row through 0 * NaN ("cuDNN Frontend v1.28.0 release notes",
 // "Updates to Graph API / SDPA", max_total_seq_len).  Fully masked KV tiles
 // past the causal diagonal are never loaded.
 #pragma once
@@ -40,15 +48,15 @@ struct PrefillParams {
     CUtensorMap tm_v;
     int mode;  // 0 dense, 1 ragged
     int B, Hq, Hkv, G;
-    int heads_per_item;  // 2 when G is even, else 1
-    int n_pairs;         // Hq / heads_per_item
-    int Sq, Skv;         // dense
-    int n_qtiles;        // dense: ceil(Sq / 128)
-    int n_items;         // dense: number of work items
+    int heads_per_item;   // 2 when G is even, else 1
+    int pairs_per_group;  // G / heads_per_item
+    int Sq, Skv;          // dense
+    int n_qtiles;         // dense: ceil(Sq / 128)
+    int n_items;          // dense: number of work items
     const int32_t* cu_q;
     const int32_t* cu_kv;
-    const int4* items;     // ragged: work list {b, qtile, h0, cost}
-    const int* n_items_dev;  // ragged: its length
+    const int4* items;  // ragged: work list {b, qtile, h0, cost}
+    int* header;        // ragged: [0] item count, [1] claim counter
     __nv_bfloat16* o;
     int64_t o_bs, o_ts, o_hs;  // element strides (batch, token, head)
     float* lse;
@@ -60,11 +68,11 @@ struct PrefillParams {
 
 struct PrefillItem {
     int b, qt, h0, nh;
-    int q_tok0;      // token coordinate of row 0 (dense: inside the batch)
-    int kv_tok0;     // token coordinate of key 0
-    int batch;       // batch coordinate (dense) or 0
+    int q_tok0;   // token coordinate of row 0 (dense: inside the batch)
+    int kv_tok0;  // token coordinate of key 0
+    int batch;    // batch coordinate (dense) or 0
     int Lq, Lkv;
-    int n_kv;        // KV tiles to visit
+    int n_kv;     // KV tiles to visit
 };
 
 __device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal) {
@@ -78,12 +86,16 @@ __device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal)
 
 __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx, PrefillItem& it) {
     if (p.mode == 0) {
-        const int per_tile = p.B * p.n_pairs;
-        const int q = idx / per_tile;
-        const int rem = idx - q * per_tile;
-        it.qt = p.causal ? (p.n_qtiles - 1 - q) : q;  // longest (latest) tiles first
-        it.b = rem / p.n_pairs;
-        it.h0 = (rem - it.b * p.n_pairs) * p.heads_per_item;
+        // dense: (batch, kv head, query tile longest first, head pair)
+        const int per_b = p.Hkv * p.n_qtiles * p.pairs_per_group;
+        it.b = idx / per_b;
+        int rem = idx - it.b * per_b;
+        const int g = rem / (p.n_qtiles * p.pairs_per_group);
+        rem -= g * p.n_qtiles * p.pairs_per_group;
+        const int t = rem / p.pairs_per_group;
+        const int pr = rem - t * p.pairs_per_group;
+        it.qt = p.causal ? (p.n_qtiles - 1 - t) : t;
+        it.h0 = g * p.G + pr * p.heads_per_item;
         it.q_tok0 = it.qt * 128;
         it.kv_tok0 = 0;
         it.batch = it.b;
@@ -111,14 +123,19 @@ struct PrefillCfg {
     static constexpr int HALVES = D / 64;
     static constexpr uint32_t TILE = HALVES * 16384u;  // one 128-row bf16 tile
     static constexpr int NST = (D == 128) ? 5 : 8;     // K/V ring depth
+    static constexpr int NRING = 2;                    // published work items in flight
     static constexpr uint32_t BAR_OFF = (2 + NST) * TILE;
     static constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
 };
+
+// Exponentials per 32-column chunk evaluated on the FMA pipe (the rest on MUFU).
+constexpr int kEmuPer32 = 0;
 
 template <int D>
 __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     using C = PrefillCfg<D>;
     constexpr int NST = C::NST;
+    constexpr int NRING = C::NRING;
     constexpr uint32_t TILE = C::TILE;
     constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, false);
     constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, true);
@@ -139,8 +156,12 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
     const uint32_t b_odone0 = b_qfull + 48;   // + 8*slot
     const uint32_t b_oempty0 = b_qfull + 64;  // + 8*slot
     const uint32_t b_drain = b_qfull + 80;
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::BAR_OFF + 16u * NST + 96);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + 16u * NST + 100);
+    const uint32_t b_ifull0 = b_qfull + 88;              // + 8*ring slot
+    const uint32_t b_iempty0 = b_ifull0 + 8 * NRING;     // + 8*ring slot
+    const uint32_t misc = 16u * NST + 88 + 16 * NRING;   // byte offset past the barriers
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::BAR_OFF + misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + misc + 4);
+    volatile int* item_ring = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + misc + 8);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -159,6 +180,10 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
             mbar_init(b_oempty0 + 8 * s, 128);
         }
         mbar_init(b_drain, 1);
+        for (int r = 0; r < NRING; ++r) {
+            mbar_init(b_ifull0 + 8 * r, 1);
+            mbar_init(b_iempty0 + 8 * r, 9);  // MMA thread + one lane of each softmax warp
+        }
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&p.tm_q);
@@ -173,13 +198,29 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    const int n_items = (p.mode == 0) ? p.n_items : *p.n_items_dev;
+
+    // Consumers read the next published item (-1 ends the loop).
+    auto next_item = [&](int k, bool arrive_lane) -> int {
+        const int r = k % NRING;
+        if (!mbar_wait(b_ifull0 + 8 * r, (k / NRING) & 1, abort_flag)) return -1;
+        const int idx = item_ring[r];
+        if (arrive_lane) mbar_arrive(b_iempty0 + 8 * r);
+        return idx;
+    };
 
     if (warp == 0 && lane == 0) {
-        // ------------------------------------------------------------ producer
+        // ---------------------------------------------- scheduler + producer
+        const int n_items = (p.mode == 0) ? p.n_items : p.header[0];
         int kv_it = 0, q_it = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            const int r = k % NRING;
+            if (!mbar_wait(b_iempty0 + 8 * r, ((k / NRING) & 1) ^ 1, abort_flag)) break;
+            int idx = (p.mode == 0) ? (int)blockIdx.x + k * (int)gridDim.x : atomicAdd(p.header + 1, 1);
+            if (idx >= n_items) idx = -1;
+            item_ring[r] = idx;
+            mbar_arrive(b_ifull0 + 8 * r);
+            if (idx < 0) break;
             PrefillItem it;
             prefill_get_item(p, idx, it);
             if (it.n_kv == 0) continue;
@@ -206,13 +247,13 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
         }
         // Let every load this thread issued land before the block exits.
         const int n_last = min(kv_it, NST);
-        for (int k = kv_it - n_last; k < kv_it; ++k)
-            mbar_wait(full_bar(k % NST), (k / NST) & 1, nullptr, 100000000ull);
+        for (int kk = kv_it - n_last; kk < kv_it; ++kk)
+            mbar_wait(full_bar(kk % NST), (kk / NST) & 1, nullptr, 100000000ull);
         if (q_it > 0) mbar_wait(b_qfull, (q_it - 1) & 1, nullptr, 100000000ull);
     } else if (warp == 1 && lane == 0) {
         // --------------------------------------------------------- MMA issuer
         int kv_it = 0, q_it = 0;
-        int pr_cnt[2] = {0, 0}, oe_cnt[2] = {0, 0};
+        int pr_cnt0 = 0, pr_cnt1 = 0, oe_cnt0 = 0, oe_cnt1 = 0;
         bool ok = true;
         auto issue_qk = [&](int s, int st) {
             const uint32_t d_tmem = tmem + 128u * s;
@@ -233,14 +274,16 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
                 tc_mma_ts(d_tmem, a_tmem + kk * 8u, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
             }
         };
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            const int idx = next_item(k, true);
+            if (idx < 0) break;
             PrefillItem it;
             prefill_get_item(p, idx, it);
             if (it.n_kv == 0) continue;
             if (!mbar_wait(b_qfull, q_it & 1, abort_flag)) { ok = false; break; }
             ++q_it;
             // prologue: S = Q K(0)^T for both slots
-            int stK = kv_it % NST;
+            const int stK = kv_it % NST;
             if (!mbar_wait(full_bar(stK), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
             ++kv_it;
             tc_fence_after();
@@ -258,11 +301,13 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
                 const int stK1 = kv_it % NST;
                 const uint32_t parK1 = (kv_it / NST) & 1;
                 for (int s = 0; ok && s < it.nh; ++s) {
-                    if (!mbar_wait(b_pready0 + 8 * s, pr_cnt[s] & 1, abort_flag)) { ok = false; break; }
-                    ++pr_cnt[s];
+                    int& pr_cnt = s ? pr_cnt1 : pr_cnt0;
+                    int& oe_cnt = s ? oe_cnt1 : oe_cnt0;
+                    if (!mbar_wait(b_pready0 + 8 * s, pr_cnt & 1, abort_flag)) { ok = false; break; }
+                    ++pr_cnt;
                     if (j == 0) {
-                        if (!mbar_wait(b_oempty0 + 8 * s, (oe_cnt[s] & 1) ^ 1, abort_flag)) { ok = false; break; }
-                        ++oe_cnt[s];
+                        if (!mbar_wait(b_oempty0 + 8 * s, (oe_cnt & 1) ^ 1, abort_flag)) { ok = false; break; }
+                        ++oe_cnt;
                     }
                     tc_fence_after();
                     issue_pv(s, stV, j > 0);
@@ -299,9 +344,15 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
         const uint32_t b_sfull = b_sfull0 + 8 * slot, b_pready = b_pready0 + 8 * slot;
         const uint32_t b_odone = b_odone0 + 8 * slot, b_oempty = b_oempty0 + 8 * slot;
         const float sl2 = p.scale_log2;
+        const bool pos = sl2 >= 0.f;  // sign of the scale decides max vs min of raw scores
+        const float NEG = pos ? -INFINITY : INFINITY;
         int sf_cnt = 0, od_base = 0;
         bool ok = true;
-        for (int idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+        for (int k = 0; ok; ++k) {
+            int idx = next_item(k, false);
+            __syncwarp();
+            if (lane == 0 && idx >= -1) mbar_arrive(b_iempty0 + 8 * (k % NRING));
+            if (idx < 0) break;
             PrefillItem it;
             prefill_get_item(p, idx, it);
             if (slot >= it.nh) continue;
@@ -319,30 +370,48 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
                     tc_fence_after();
                     float x[128];
                     {
-                        uint32_t u[32];
+                        uint32_t u0[32], u1[32], u2[32], u3[32];
+                        tmem_ld32(tS, u0);
+                        tmem_ld32(tS + 32u, u1);
+                        tmem_ld32(tS + 64u, u2);
+                        tmem_ld32(tS + 96u, u3);
+                        tc_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            tmem_ld32(tS + 32u * c, u);
-                            tc_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) x[32 * c + e] = __uint_as_float(u[e]);
+                        for (int e = 0; e < 32; ++e) {
+                            x[e] = __uint_as_float(u0[e]);
+                            x[32 + e] = __uint_as_float(u1[e]);
+                            x[64 + e] = __uint_as_float(u2[e]);
+                            x[96 + e] = __uint_as_float(u3[e]);
                         }
                     }
                     const int kb = j * 128;
-                    float mx = -INFINITY;
-                    if (kb + 128 > lim) {
+                    const bool masked = (kb + 128 > lim);
+                    if (masked) {
 #pragma unroll
-                        for (int c = 0; c < 128; ++c) {
-                            x[c] = (kb + c < lim) ? x[c] * sl2 : -INFINITY;
-                            mx = fmaxf(mx, x[c]);
+                        for (int c = 0; c < 128; ++c) x[c] = (kb + c < lim) ? x[c] : NEG;
+                    }
+                    // row maximum of the scaled scores (min of raw scores when scale < 0)
+                    float a0 = NEG, a1 = NEG, a2 = NEG, a3 = NEG;
+                    if (pos) {
+#pragma unroll
+                        for (int c = 0; c < 128; c += 8) {
+                            a0 = fmax3(a0, x[c], x[c + 1]);
+                            a1 = fmax3(a1, x[c + 2], x[c + 3]);
+                            a2 = fmax3(a2, x[c + 4], x[c + 5]);
+                            a3 = fmax3(a3, x[c + 6], x[c + 7]);
                         }
+                        a0 = fmax3(a0, a1, fmaxf(a2, a3));
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 128; ++c) {
-                            x[c] *= sl2;
-                            mx = fmaxf(mx, x[c]);
+                        for (int c = 0; c < 128; c += 8) {
+                            a0 = fmin3(a0, x[c], x[c + 1]);
+                            a1 = fmin3(a1, x[c + 2], x[c + 3]);
+                            a2 = fmin3(a2, x[c + 4], x[c + 5]);
+                            a3 = fmin3(a3, x[c + 6], x[c + 7]);
                         }
+                        a0 = fmin3(a0, a1, fminf(a2, a3));
                     }
+                    const float mx = (a0 == NEG) ? -INFINITY : a0 * sl2;
                     const float m_new = fmaxf(m_use, mx);
                     float alpha = 1.f;
                     const bool old_finite = (m_use != -INFINITY);
@@ -351,20 +420,34 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
                         m_use = m_new;
                     }
                     const float mref = (m_use == -INFINITY) ? 0.f : m_use;
-                    float sum = 0.f;
+                    const float2 sc2 = make_float2(sl2, sl2);
+                    const float2 nm2 = make_float2(-mref, -mref);
+                    float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t pk[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
-                            const float p0 = ex2(x[32 * c + 2 * e] - mref);
-                            const float p1 = ex2(x[32 * c + 2 * e + 1] - mref);
-                            sum += p0 + p1;
-                            pk[e] = pack_bf16(p0, p1);
+                            const int col = 32 * c + 2 * e;
+                            const float2 t = ffma2(make_float2(x[col], x[col + 1]), sc2, nm2);
+                            float2 pv;
+                            if (2 * e >= 32 - kEmuPer32) {
+                                pv = exp2_poly_pair(t);
+                            } else {
+                                pv.x = ex2(t.x);
+                                pv.y = ex2(t.y);
+                            }
+                            if (masked) {
+                                pv.x = (kb + col < lim) ? pv.x : 0.f;
+                                pv.y = (kb + col + 1 < lim) ? pv.y : 0.f;
+                            }
+                            if (e & 1) sum1 = fadd2(sum1, pv);
+                            else sum0 = fadd2(sum0, pv);
+                            pk[e] = pack_bf16(pv.x, pv.y);
                         }
                         tmem_st16(tS + 16u * c, pk);
                     }
-                    l = l * alpha + sum;
+                    l = l * alpha + ((sum0.x + sum0.y) + (sum1.x + sum1.y));
                     const bool need_o = (j > 0) && old_finite && (alpha != 1.f);
                     if (__any_sync(0xffffffffu, need_o)) {
                         // PV(j-1) must have landed in O before it is rescaled.

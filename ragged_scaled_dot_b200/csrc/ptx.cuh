@@ -214,6 +214,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | ((uint32_t)(M >> 4) << 24);
 }
 
+// Per-warpgroup register reallocation.  All four warps of a warpgroup must
+// execute the same instruction, and the block's total (threads x registers)
+// must not exceed what it was launched with.
+template <int N>
+__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // ---------------------------------------------------------------------------
 // Math helpers
 // ---------------------------------------------------------------------------
@@ -221,6 +229,57 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Packed fp32 pair arithmetic (sm_100): two lanes of work per instruction.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)),
+          "l"(*reinterpret_cast<unsigned long long*>(&c)));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(*reinterpret_cast<unsigned long long*>(&d))
+        : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+    return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^t for a pair, on the FMA pipe instead of the MUFU unit.  Base-2
+// Cody-Waite style reduction: n = round(t) by adding 1.5*2^23, f = t - n in
+// [-1/2, 1/2]; 2^f from a degree-3 polynomial we fitted by linear-programming
+// minimax of the relative error with p(0) = 1 held exact (so 2^n is exact for
+// integer t); max relative error 1.01e-4 on [-1/2, 1/2]; 2^n is applied by
+// adding n to the exponent field.  t is clamped at -125 so the result stays a
+// normal float; callers that need an exact zero (masked keys) select it.
+__device__ __forceinline__ float2 exp2_poly_pair(float2 t) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    t.x = fmaxf(t.x, -125.0f);
+    t.y = fmaxf(t.y, -125.0f);
+    const float2 j = fadd2(t, make_float2(kRound, kRound));
+    const float2 n = fadd2(j, make_float2(-kRound, -kRound));
+    const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), t);
+    float2 p = ffma2(make_float2(0.055008936673402786f, 0.055008936673402786f), f,
+                     make_float2(0.24221095442771912f, 0.24221095442771912f));
+    p = ffma2(p, f, make_float2(0.6932829022407532f, 0.6932829022407532f));
+    p = ffma2(p, f, make_float2(1.0f, 1.0f));
+    const uint32_t kBias = __float_as_uint(kRound) << 23;
+    const uint32_t ex = (__float_as_uint(j.x) << 23) - kBias;
+    const uint32_t ey = (__float_as_uint(j.y) << 23) - kBias;
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + ex), __uint_as_float(__float_as_uint(p.y) + ey));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

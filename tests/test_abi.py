@@ -47,9 +47,10 @@ def test_status_strings(lib):
 
 
 def test_workspace_sizes(lib):
-    # ragged: header + one 16-byte item per (query tile, head group)
+    # ragged: header + one 16-byte item per (query tile, head pair) + two ints per sequence
     n = rsd.attn_fwd_ragged_workspace_size(2, 64, 101, 4, 1)
-    assert n == 256 + min(101 // 128 + 2, 2 * 1) * 2 * 16
+    tiles = min(101 // 128 + 2, 2 * 1)
+    assert n >= 256 + tiles * 2 * 16 + 2 * 2 * 4 and n % 256 == 0
     assert rsd.attn_fwd_ragged_workspace_size(0, 64, 101, 4, 1) == 0
     # paged: none for one split; partial O (fp32) + partial LSE otherwise
     assert rsd.attn_fwd_paged_workspace_size(128, 64, 128, 1) == 0

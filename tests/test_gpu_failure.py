@@ -57,3 +57,22 @@ def test_out_of_range_page_id_is_reported():
     o, lse = paged_gpu(q, k, k, table, np.array(lens, np.int32), ps, 0.1, 1)
     assert rsd.attn_get_device_error() == rsd.ATTN_ERR_DEVICE_INPUT
     assert torch.isfinite(o.float()).all()
+
+
+def test_fma_pipe_exp2_error_bound():
+    """The softmax's FMA-pipe exponential against 2^t in float64: relative error
+    <= 1.1e-4 on the range the softmax uses ([-125, 8]), exact at integers
+    (so a constant score row sums to an exact count), monotone input clamp."""
+    t = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001), torch.arange(-125, 9, dtype=torch.float32),
+                   torch.tensor([-200.0, -1e30])]).to(DEV)
+    y = torch.empty_like(t)
+    rsd.attn_selftest_exp2(t, y)
+    torch.cuda.synchronize()
+    tt = t.double().cpu().numpy()
+    yy = y.double().cpu().numpy()
+    ref = np.exp2(np.maximum(tt, -125.0))
+    rel = np.abs(yy - ref) / ref
+    assert rel.max() <= 1.1e-4, rel.max()
+    ints = np.arange(-125, 9)
+    n0 = 1_000_001
+    assert np.array_equal(yy[n0:n0 + len(ints)], np.exp2(ints.astype(np.float64)))
