@@ -37,11 +37,12 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill attention TFLOPS and paged-decode KV GB/s, % of B200 roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) per algorithmic unit from the latest ncu capture of
-# each kernel (profiles/), scaled to a full launch by units processed.  None
-# when the kernel changed after the counters were taken.
-#   paged_decode: profiles/decode_gqa_kernel_paged_b32.md (2.692 GB / 2.673 GB)
-TRAFFIC_PER_UNIT = {"ragged_prefill": None, "paged_decode": 1.0071}
+# DRAM bytes (read + write) from the latest ncu capture of each kernel
+# (profiles/), as a ratio to the bytes that scale with the launch, applied to
+# the full launch.  None when the kernel changed after the counters were taken.
+#   paged_decode: per K/V byte, profiles/decode_gqa_kernel_paged_b32.md (2.692 / 2.673 GB)
+#   ragged_prefill: per Q+K+V+O byte, profiles/prefill_kernel_ragged_b16.md (1.042 / 1.061 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.982, "paged_decode": 1.0071}
 
 
 def load_peaks():
@@ -187,9 +188,11 @@ def make_ragged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
         return e2e_step, h2d, d2h
 
     flops = prefill_flops(L, L, w.Hq, w.Dqk)
+    io_gb = T * (2 * w.Hq * w.Dqk + w.Hkv * (w.Dqk + w.Dv)) * 2 / 1e9
     info = {"workload": w.notes, "B": w.B, "total_tokens": int(T), "max_seqlen": smax,
             "Hq": w.Hq, "Hkv": w.Hkv, "D": w.Dqk, "flop_per_step": flops,
-            "flop_per_unit": "4*D per visible (query, key) pair per query head"}
+            "flop_per_unit": "4*D per visible (query, key) pair per query head",
+            "traffic_basis_gb": io_gb}
     data = dict(q=q, k=k, v=v, cu=cu, L=L, w=w)
     return Part("ragged_prefill", "TFLOP/s", flops / 1e12, 3, step, e2e_setup, info), data
 
@@ -255,7 +258,7 @@ def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
 
     nbytes = decode_kv_bytes(L, w.Hkv, w.Dqk, Dv, w.v_aliases_k)
     flops = float(np.sum(L)) * w.Hq * 2.0 * (w.Dqk + Dv)
-    info = {"workload": w.notes, "num_splits": S, "kv_bytes_per_step": nbytes,
+    info = {"workload": w.notes, "num_splits": S, "kv_bytes_per_step": nbytes, "traffic_basis_gb": nbytes / 1e9,
             "flop_per_step": flops, "total_pages": int(kp.shape[0]),
             "bytes_per_unit": f"{w.Hkv * (w.Dqk if w.v_aliases_k else w.Dqk + Dv) * 2} B of K/V per cached token"}
     data = dict(q=q, kp=kp, vp=vp, table=table, L=L, w=w, S=S)
@@ -425,20 +428,20 @@ def run_ours(args):
         if bound == "tensor":
             achieved = part.units / (kern_ms / 1e3)
             peak = peaks["bf16_tflops"]
-            tpu = TRAFFIC_PER_UNIT.get(part.name)
+            tpu = TRAFFIC_RATIO.get(part.name)
             roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                     "frac": round(achieved / peak, 4),
-                    "traffic": None if tpu is None else round(part.units * tpu, 3),
+                    "traffic": None if tpu is None else round(part.info["traffic_basis_gb"] * tpu, 3),
                     "traffic_unit": "GB per launch (dram read + write)",
                     "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
                     "peak_source": f"{peak_src} bf16_tflops (burst)"}
         else:
             achieved = part.units / (kern_ms / 1e3)
             peak = peaks["hbm_gbs"]
-            tpu = TRAFFIC_PER_UNIT.get(part.name)
+            tpu = TRAFFIC_RATIO.get(part.name)
             roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4),
-                    "traffic": None if tpu is None else round(part.units * tpu, 3),
+                    "traffic": None if tpu is None else round(part.info["traffic_basis_gb"] * tpu, 3),
                     "traffic_unit": "GB per launch (dram read + write)",
                     "peak_source": f"{peak_src} hbm_gbs"}
         return value, ms, roof

@@ -13,7 +13,10 @@
 //   warp 0      claims items, publishes them to the other roles through a
 //               small shared-memory ring, and issues the TMA loads: Q tiles of
 //               the item, then K(j), V(j) into a ring of NST stages.
-//   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit.
+//   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit
+//               (descriptor bases are precomputed: this thread shares its SM
+//               sub-partition with two busy softmax warps, so every instruction
+//               it issues is expensive).
 //   warps 4-7   softmax for slot 0 (query head h0), one TMEM lane (row) each.
 //   warps 8-11  softmax for slot 1 (query head h0 + 1).
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
@@ -26,10 +29,11 @@
 // runs.  The softmax keeps the running maximum m in the log2 domain with the
 // scale folded in ("cuDNN Frontend v1.30.0 Release Notes", stats_use_log2
 // section: the prefill kernels keep the softmax in the log2 domain), only
-// rescales O when the maximum grows by more than 8 (P stays <= 2^8), and
-// evaluates part of the exponentials on the FMA pipe so the MUFU unit is not
-// the only source ("cuDNN Frontend v1.30.0 Release Notes", "SDPA: more kernels
-// and numerics": exp2 on the FMA pipe).
+// rescales O when the maximum grows by more than 8 (P stays <= 2^8).  An
+// FMA-pipe exponential ("cuDNN Frontend v1.30.0 Release Notes", "SDPA: more
+// kernels and numerics": exp2 on the FMA pipe) is available through
+// kEmuPer32 but measured slower here, so it is off: with one softmax warp per
+// sub-partition the exponential loop is latency-bound, not MUFU-bound.
 //
 // Masking: bottom-right causal per sequence and ragged tails are applied by
 // select, never by multiplication, so values past a sequence's end can not
@@ -255,23 +259,26 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
         int kv_it = 0, q_it = 0;
         int pr_cnt0 = 0, pr_cnt1 = 0, oe_cnt0 = 0, oe_cnt1 = 0;
         bool ok = true;
+        const SmemDesc dQ = smem_desc_sw128_split(sQ, 16, 1024);
+        const SmemDesc dK = smem_desc_sw128_split(sKV, 16, 1024);
+        const SmemDesc dV = smem_desc_sw128_split(sKV, 16384, 1024);
         auto issue_qk = [&](int s, int st) {
             const uint32_t d_tmem = tmem + 128u * s;
+            const SmemDesc a0{dQ.lo + ((s * TILE) >> 4), dQ.hi};
+            const SmemDesc b0{dK.lo + ((st * TILE) >> 4), dK.hi};
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                const uint64_t a = smem_desc_sw128(sQ + s * TILE + off, 16, 1024);
-                const uint64_t b = smem_desc_sw128(sKV + st * TILE + off, 16, 1024);
-                tc_mma_ss(d_tmem, a, b, IDESC_QK, kk > 0 ? 1u : 0u);
+                tc_mma_ss(d_tmem, desc_at(a0, off), desc_at(b0, off), IDESC_QK, kk > 0 ? 1u : 0u);
             }
         };
         auto issue_pv = [&](int s, int st, bool acc) {
             const uint32_t d_tmem = tmem + 256u + (uint32_t)(D * s);
             const uint32_t a_tmem = tmem + 128u * s;
+            const SmemDesc b0{dV.lo + ((st * TILE) >> 4), dV.hi};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t b = smem_desc_sw128(sKV + st * TILE + kk * 2048u, 16384, 1024);
-                tc_mma_ts(d_tmem, a_tmem + kk * 8u, b, IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                tc_mma_ts(d_tmem, a_tmem + kk * 8u, desc_at(b0, kk * 2048u), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
             }
         };
         for (int k = 0; ok; ++k) {

@@ -203,6 +203,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
     return d;
 }
 
+// The same descriptor split in halves: the low word holds the start address
+// (>> 4) and the leading byte offset, the high word the stride byte offset,
+// version and swizzle.  Advancing a descriptor by `bytes` (16-byte multiple,
+// staying inside shared memory) is one 32-bit add on the low word.
+struct SmemDesc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ SmemDesc smem_desc_sw128_split(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    const uint64_t d = smem_desc_sw128(addr, lbo_bytes, sbo_bytes);
+    return SmemDesc{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+__device__ __forceinline__ uint64_t desc_at(SmemDesc d, uint32_t bytes) {
+    return ((uint64_t)d.hi << 32) | (uint64_t)(d.lo + (bytes >> 4));
+}
+
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulation.
 // b_mn_major: B operand stored MN-major (N contiguous) instead of K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
