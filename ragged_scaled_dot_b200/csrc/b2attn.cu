@@ -15,6 +15,7 @@
 #include "prefill.cuh"
 #include "aux_kernels.cuh"
 #include "decode.cuh"
+#include "decode_mla.cuh"
 
 namespace {
 
@@ -68,11 +69,8 @@ int setup_device(int* dev_out, int* sms_out) {
             e = cudaFuncSetAttribute(b2::decode_gqa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::DecodeCfg<128>::SMEM);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(b2::decode_mla_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     b2::MlaCfg<true>::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(b2::decode_mla_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     b2::MlaCfg<false>::SMEM);
+            e = cudaFuncSetAttribute(b2::decode_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::MlaTcCfg::SMEM);
         if (e != cudaSuccess) return ATTN_ERR_CUDA;
         st.num_sms = sms;
         st.ready = true;
@@ -405,10 +403,9 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     const bool mla = (Dqk == 576 && Dv == 512);
     const bool gqa = (Dqk == Dv && (Dqk == 64 || Dqk == 128) && G <= 16);
     if (!mla && !gqa) return ATTN_ERR_UNSUPPORTED;
-    if (mla && (Hkv != 1 || Hq % 64 != 0)) return ATTN_ERR_UNSUPPORTED;
-    // a 64-key chunk is whole pages, or a page is whole chunks
+    if (mla && Hkv != 1) return ATTN_ERR_UNSUPPORTED;
+    // a 64-key box is whole pages, or a page is whole boxes
     if (!(page_size % 64 == 0 || (64 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
-    if (mla && !(page_size % 32 == 0 || (32 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
     if (B == 0) return ATTN_OK;
     if (!q || !k_pool || !v_pool || !o || !page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
@@ -428,13 +425,11 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     int dev, sms;
     if (int e = setup_device(&dev, &sms)) return e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool alias = mla && (v_pool == k_pool) && std::memcmp(k_pool_strides, v_pool_strides, 3 * sizeof(int64_t)) == 0;
 
     DecodeParams dp;
     std::memset(&dp, 0, sizeof(dp));
-    // rows per TMA box: one page, at most one chunk (64 keys GQA, 32 keys MLA)
-    const int chunk_keys = mla ? 32 : 64;
-    const int box_rows = page_size < chunk_keys ? page_size : chunk_keys;
+    // rows per TMA box: one page, at most 64 keys
+    const int box_rows = page_size < 64 ? page_size : 64;
     {
         const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
         const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
@@ -443,12 +438,6 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
         const uint64_t dv[4] = {(uint64_t)Dv, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
         const int64_t sv[3] = {v_pool_strides[1], v_pool_strides[2], v_pool_strides[0]};
         if (encode_4d(&dp.tm_v, v_pool, dv, sv, box)) return ATTN_ERR_INVALID_ARG;
-        if (mla) {
-            const uint32_t qbox[4] = {64, 64, 1, 1};
-            const uint64_t dq[4] = {(uint64_t)Dqk, (uint64_t)Hq, (uint64_t)B, 1};
-            const int64_t sq[3] = {q_strides[1], q_strides[0], unit_dim_stride(q_strides[0] * B, 8)};
-            if (encode_4d(&dp.tm_q, q, dq, sq, qbox)) return ATTN_ERR_INVALID_ARG;
-        }
     }
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.q_bs = q_strides[0];
@@ -477,11 +466,23 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
                                                round_up(R * num_splits * Dv * 4, 256));
     }
     if (mla) {
-        dim3 grid(num_splits, Hq / 64, B);
-        if (alias)
-            b2::decode_mla_kernel<true><<<grid, 288, b2::MlaCfg<true>::SMEM, st>>>(dp);
-        else
-            b2::decode_mla_kernel<false><<<grid, 288, b2::MlaCfg<false>::SMEM, st>>>(dp);
+        // one cluster of two CTAs (score CTA, value CTA) per (b, split, group of 128 heads)
+        const int64_t units = (int64_t)B * num_splits * ((Hq + 127) / 128);
+        if (2 * units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
+        cfg.blockDim = dim3(b2::MlaTcCfg::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = b2::MlaTcCfg::SMEM;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, b2::decode_mla_tc_kernel, dp) != cudaSuccess) return ATTN_ERR_LAUNCH;
     } else {
         dim3 grid(num_splits, Hkv, B);
         if (Dqk == 128)

@@ -23,7 +23,6 @@ namespace b2 {
 struct DecodeParams {
     CUtensorMap tm_k;  // 4D (d, slot, head, page), 128B swizzle, box (64, min(ps,64), 1, 1)
     CUtensorMap tm_v;
-    CUtensorMap tm_q;  // MLA only: 3D (d, head, batch), box (64, 64, 1)
     const __nv_bfloat16* q;
     int64_t q_bs, q_hs;
     const int32_t* page_table;
@@ -334,260 +333,6 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
         }
     }
     (void)ok;
-    __syncthreads();
-}
-
-// ===========================================================================
-// Absorbed-MLA decode: Dqk = 576, Dv = 512, every query head shares one KV
-// head ("cuDNN Frontend v1.32.0 Release Notes", "SDPA: wider native forward
-// support").  grid (num_splits, Hq / 64, B); 288 threads: warps 0-7 compute,
-// warp 8 loads.  Warp w covers query heads [16*(w/2), +16) of the block's 64
-// and value columns [256*(w%2), +256); both warps of a pair compute the same
-// scores.  With V aliasing K, V is read from the K tile already in shared
-// memory.  Chunks are 32 keys.
-// ===========================================================================
-template <bool ALIAS>
-struct MlaCfg {
-    static constexpr int DQK = 576, DV = 512;
-    static constexpr int KEYS = 32;
-    static constexpr uint32_t KBLK = KEYS * 128;         // 32 rows x 128 B
-    static constexpr uint32_t KCHUNK = 9 * KBLK;         // 36 KB
-    static constexpr uint32_t VCHUNK = ALIAS ? 0 : 8 * KBLK;
-    static constexpr uint32_t STAGE = KCHUNK + VCHUNK;
-    static constexpr int NST = ALIAS ? 3 : 2;
-    static constexpr uint32_t QBLK = 64 * 128;           // 64 heads x 128 B
-    static constexpr uint32_t QBYTES = 9 * QBLK;         // 72 KB
-    static constexpr uint32_t RING_OFF = QBYTES;
-    static constexpr uint32_t BAR_OFF = RING_OFF + NST * STAGE;
-    static constexpr uint32_t SMEM = BAR_OFF + 128 + 1024;
-};
-
-template <bool ALIAS>
-__global__ void __launch_bounds__(288, 1) decode_mla_kernel(const __grid_constant__ DecodeParams p) {
-    using C = MlaCfg<ALIAS>;
-    constexpr int NST = C::NST;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t sb = (raw + 1023u) & ~1023u;
-    uint8_t* sgen = smem_raw + (sb - raw);
-    const uint32_t sQ = sb;
-    const uint32_t sRing = sb + C::RING_OFF;
-    const uint32_t sBar = sb + C::BAR_OFF;
-    auto full_bar = [&](int i) { return sBar + 8u * i; };
-    auto empty_bar = [&](int i) { return sBar + 8u * (NST + i); };
-    const uint32_t b_q = sBar + 16u * NST;
-    const uint32_t b_tail = b_q + 8;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + 16u * NST + 16);
-
-    const int s = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    int L, lo, hi;
-    decode_split_range(p, b, s, L, lo, hi);
-    const int n_chunks = (hi > lo) ? (hi - lo + C::KEYS - 1) / C::KEYS : 0;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < NST; ++i) {
-            mbar_init(full_bar(i), 1);
-            mbar_init(empty_bar(i), 8);
-        }
-        mbar_init(b_q, 1);
-        mbar_init(b_tail, 1);
-        *abort_flag = 0;
-        fence_barrier_init();
-    }
-    __syncthreads();
-
-    if (warp == 8) {
-        if (lane == 0) {
-            prefetch_tmap(&p.tm_k);
-            prefetch_tmap(&p.tm_q);
-            mbar_arrive_expect_tx(b_q, C::QBYTES);
-            for (int cb = 0; cb < 9; ++cb) tma_load_4d(sQ + cb * C::QBLK, &p.tm_q, b_q, cb * 64, hg * 64, b, 0);
-            for (int c = 0; c < n_chunks; ++c) {
-                const int st = c % NST;
-                if (!mbar_wait(empty_bar(st), ((c / NST) & 1) ^ 1, abort_flag)) break;
-                const int t0 = lo + c * C::KEYS;
-                const int nkeys = min(C::KEYS, hi - t0);
-                const int nboxes = (nkeys + p.box_rows - 1) / p.box_rows;
-                const uint32_t kbytes = (uint32_t)nboxes * p.box_rows * 128u * 9u;
-                const uint32_t vbytes = ALIAS ? 0u : (uint32_t)nboxes * p.box_rows * 128u * 8u;
-                mbar_arrive_expect_tx(full_bar(st), kbytes + vbytes);
-                const uint32_t dst = sRing + st * C::STAGE;
-                for (int r = 0; r < nkeys; r += p.box_rows) {
-                    const int t = t0 + r;
-                    int page = __ldg(p.page_table + (int64_t)b * p.pt_stride + t / p.page_size);
-                    if (page < 0 || (int64_t)page >= p.num_pages) {
-                        record_status(ATTN_ERR_DEVICE_INPUT);
-                        page = -1;
-                    }
-                    const int slot = t % p.page_size;
-                    for (int cb = 0; cb < 9; ++cb)
-                        tma_load_4d(dst + cb * C::KBLK + r * 128u, &p.tm_k, full_bar(st), cb * 64, slot, 0, page);
-                    if (!ALIAS)
-                        for (int cb = 0; cb < 8; ++cb)
-                            tma_load_4d(dst + C::KCHUNK + cb * C::KBLK + r * 128u, &p.tm_v, full_bar(st),
-                                        cb * 64, slot, 0, page);
-                }
-                if (nkeys < C::KEYS) {
-                    // The one partial chunk: once it lands, zero the value rows past the
-                    // sequence (aliased: the K rows) so 0 * (stale or NaN) never reaches O,
-                    // then release it to the compute warps through b_tail.
-                    if (!mbar_wait(full_bar(st), (c / NST) & 1, abort_flag)) break;
-                    uint8_t* vg = sgen + ((ALIAS ? dst : dst + C::KCHUNK) - sb);
-                    for (int rr = nkeys; rr < C::KEYS; ++rr)
-                        for (int i = 0; i < 8 * 8; ++i)
-                            *reinterpret_cast<uint4*>(vg + (i >> 3) * C::KBLK + rr * 128 + (i & 7) * 16) =
-                                make_uint4(0, 0, 0, 0);
-                    mbar_arrive(b_tail);
-                }
-            }
-            for (int c = max(0, n_chunks - NST); c < n_chunks; ++c)
-                mbar_wait(full_bar(c % NST), (c / NST) & 1, nullptr, 100000000ull);
-            mbar_wait(b_q, 0, nullptr, 100000000ull);
-        }
-        __syncthreads();
-        return;
-    }
-
-    const float sl2 = p.scale_log2;
-    const int mt = warp >> 1, dh = warp & 1;
-    const int hrow0 = mt * 16;  // first head row (within the block's 64) of this warp
-    const int qrow = lane >> 2;
-    float m[2] = {-INFINITY, -INFINITY};
-    float l[2] = {0.f, 0.f};
-    float oacc[32][4];  // 16 heads x 256 value columns
-#pragma unroll
-    for (int i = 0; i < 32; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-    bool ok = mbar_wait(b_q, 0, abort_flag);
-
-    for (int c = 0; ok && c < n_chunks; ++c) {
-        const int st = c % NST;
-        if (!mbar_wait(full_bar(st), (c / NST) & 1, abort_flag)) { ok = false; break; }
-        const uint32_t sK = sRing + st * C::STAGE;
-        const uint32_t sV = ALIAS ? sK : sK + C::KCHUNK;
-        const int nvalid = min(C::KEYS, hi - (lo + c * C::KEYS));
-        if (nvalid < C::KEYS && !mbar_wait(b_tail, 0, abort_flag)) { ok = false; break; }
-        // S = Q K^T: 16 heads x 32 keys (4 n-tiles), full 576 depth
-        float sacc[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-        {
-            const int mat = lane >> 3, rr = lane & 7;
-#pragma unroll 4
-            for (int kk = 0; kk < 36; ++kk) {
-                const int cb = kk >> 2;
-                uint32_t a[4];
-                {
-                    // A (16 x 16) from Q: matrices (rows 0-7,k0-7) (rows 8-15,k0-7) (rows 0-7,k8-15) (rows 8-15,k8-15)
-                    const int row = hrow0 + ((mat & 1) << 3) + rr;
-                    const int dcol = (kk & 3) * 16 + ((mat >> 1) << 3);
-                    ldsm_x4(sQ + cb * C::QBLK + sw128_offset(row, dcol), a[0], a[1], a[2], a[3]);
-                }
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    const int key = np * 16 + ((mat >> 1) << 3) + rr;
-                    const int dcol = (kk & 3) * 16 + ((mat & 1) << 3);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(sK + cb * C::KBLK + sw128_offset(key, dcol), b0, b1, b2, b3);
-                    mma_bf16_16816(sacc[2 * np], a, b0, b1);
-                    mma_bf16_16816(sacc[2 * np + 1], a, b2, b3);
-                }
-            }
-        }
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = nt * 8 + 2 * (lane & 3) + (e & 1);
-                const float x = (key < nvalid) ? sacc[nt][e] * sl2 : -INFINITY;
-                sacc[nt][e] = x;
-                mx[e >> 1] = fmaxf(mx[e >> 1], x);
-            }
-        float alpha[2], mref[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
-            mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-            const float mn = fmaxf(m[h], mx[h]);
-            alpha[h] = (m[h] == -INFINITY) ? 0.f : ex2(m[h] - mn);
-            m[h] = mn;
-            mref[h] = (mn == -INFINITY) ? 0.f : mn;
-        }
-        float psum[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float pv = ex2(sacc[nt][e] - mref[e >> 1]);
-                sacc[nt][e] = pv;
-                psum[e >> 1] += pv;
-            }
-        l[0] = l[0] * alpha[0] + psum[0];
-        l[1] = l[1] * alpha[1] + psum[1];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            oacc[i][0] *= alpha[0];
-            oacc[i][1] *= alpha[0];
-            oacc[i][2] *= alpha[1];
-            oacc[i][3] *= alpha[1];
-        }
-        // O += P V: k = 32 keys (2 k-steps), n = 256 value columns (32 n-tiles)
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            uint32_t pa[4];
-            pa[0] = pack_bf16(sacc[2 * ks][0], sacc[2 * ks][1]);
-            pa[1] = pack_bf16(sacc[2 * ks][2], sacc[2 * ks][3]);
-            pa[2] = pack_bf16(sacc[2 * ks + 1][0], sacc[2 * ks + 1][1]);
-            pa[3] = pack_bf16(sacc[2 * ks + 1][2], sacc[2 * ks + 1][3]);
-            const int mat = lane >> 3, rr = lane & 7;
-            const int key = ks * 16 + ((mat & 1) << 3) + rr;
-#pragma unroll
-            for (int nd = 0; nd < 16; ++nd) {
-                const int vcol = dh * 256 + nd * 16;
-                const int cb = vcol >> 6;
-                const int dcol = (vcol & 63) + ((mat >> 1) << 3);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(sV + cb * C::KBLK + sw128_offset(key, dcol), v0, v1, v2, v3);
-                mma_bf16_16816(oacc[2 * nd], pa, v0, v1);
-                mma_bf16_16816(oacc[2 * nd + 1], pa, v2, v3);
-            }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(st));
-    }
-
-    // epilogue: each warp owns complete rows for its 256 value columns
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 1);
-        l[h] += __shfl_xor_sync(0xffffffffu, l[h], 2);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int head = hg * 64 + hrow0 + qrow + 8 * h;
-        const float inv = (l[h] > 0.f) ? 1.f / l[h] : 0.f;
-        const float lse = (l[h] > 0.f) ? (m[h] + log2f(l[h])) * 0.6931471805599453f : -INFINITY;
-        if (p.num_splits == 1) {
-            __nv_bfloat16* orow = p.o + (int64_t)b * p.o_bs + (int64_t)head * p.o_hs;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int col = dh * 256 + i * 8 + 2 * (lane & 3);
-                *reinterpret_cast<uint32_t*>(orow + col) = pack_bf16(oacc[i][2 * h] * inv, oacc[i][2 * h + 1] * inv);
-            }
-            if (dh == 0 && (lane & 3) == 0 && p.lse != nullptr) p.lse[(int64_t)b * p.Hq + head] = lse;
-        } else {
-            const int64_t rr = (int64_t)s * p.B * p.Hq + (int64_t)b * p.Hq + head;
-            float* orow = p.o_part + rr * C::DV;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int col = dh * 256 + i * 8 + 2 * (lane & 3);
-                *reinterpret_cast<float2*>(orow + col) = make_float2(oacc[i][2 * h] * inv, oacc[i][2 * h + 1] * inv);
-            }
-            if (dh == 0 && (lane & 3) == 0) p.lse_part[rr] = lse;
-        }
-    }
     __syncthreads();
 }
 

@@ -72,18 +72,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test with cluster-scope acquire: for barriers that a peer CTA of the
+// cluster arrives on, so its writes before the arrival are visible here.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Bounded: gives up
 // after `limit_ns` (or as soon as *abort is set by another role of the block),
 // records ATTN_ERR_DEVICE_TIMEOUT, sets *abort and returns false.
+template <bool kClusterScope = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                           unsigned long long limit_ns = kWaitLimitNs) {
+    auto test = [&]() { return kClusterScope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
 #pragma unroll 1
     for (int i = 0; i < 256; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+        if (test()) return true;
     const unsigned long long t0 = globaltimer();
 #pragma unroll 1
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (test()) return true;
         if (abort != nullptr && *abort) return false;
         if (globaltimer() - t0 > limit_ns) {
             record_status(ATTN_ERR_DEVICE_TIMEOUT);
@@ -91,6 +107,67 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
             return false;
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, the cluster-wide barrier, addresses in a peer
+// CTA's shared memory, arrivals on a peer's mbarrier, and bulk copies from this
+// CTA's shared memory into a peer's (completion counted on the peer's barrier).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address, in the cluster shared window, of `local` in the CTA of rank `rank`.
+__device__ __forceinline__ uint32_t peer_smem(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_peer(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+                 "r"(bytes)
+                 : "memory");
+}
+// bytes (multiple of 16) from this CTA's shared memory at src to dst in the
+// cluster window; both 16-byte aligned.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t cluster_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst_cluster),
+        "r"(src), "r"(bytes), "r"(cluster_bar)
+        : "memory");
+}
+
+// Named-barrier reductions over `count` threads (a multiple of 32, every
+// thread of each participating warp): all wait, all get the AND / OR.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool v) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out)
+        : "r"(v ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return out != 0;
+}
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t count, bool v) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(out)
+        : "r"(v ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return out != 0;
 }
 
 // ---------------------------------------------------------------------------

@@ -118,6 +118,96 @@ def test_mla_nan_past_kv_len_aliased():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+MLA_CASES = [
+    # (lens, Hq, ps, splits, alias): chunk edges, padded head groups, page sizes
+    ([1, 127, 128, 129, 300], 64, 64, 1, True),
+    ([257, 1000], 192, 64, 2, True),
+    ([500, 77], 128, 16, 1, False),
+    ([600, 130], 128, 128, 3, True),
+    ([3000], 16, 32, 5, True),
+    ([2, 64, 65], 128, 8, 2, False),
+]
+
+
+@pytest.mark.parametrize("lens,Hq,ps,splits,alias", MLA_CASES)
+def test_mla_decode_shapes(lens, Hq, ps, splits, alias):
+    q, k, v, table, kl = _paged_inputs(lens, Hq, 1, 576, ps, seed=31 + ps + Hq, Dv=512, alias=alias)
+    check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(576), splits, Dv=512,
+                where=f"mla {lens} Hq{Hq} ps{ps} S{splits} alias={alias}")
+
+
+def _ramp_keys(k, table, lens, ps, gain):
+    """Scale the K row of logical key j by 1 + gain*j/L, so every sequence's
+    scores keep growing and the running maximum moves many times."""
+    k = k.clone()
+    for b, L in enumerate(lens):
+        j = np.arange(L)
+        pages = torch.as_tensor(table[b, j // ps].astype(np.int64), device=DEV)
+        slots = torch.as_tensor(j % ps, device=DEV)
+        f = torch.as_tensor(1.0 + gain * j / max(L, 1), dtype=torch.float32, device=DEV)
+        rows = k[pages, 0, slots].float() * f[:, None]
+        k[pages, 0, slots] = rows.to(k.dtype)
+    return k
+
+
+@pytest.mark.parametrize("scale", [0.3, -0.3])
+def test_mla_rescale_path(scale):
+    """Scores that grow along the sequence force O rescales in the value CTA
+    (the running max rises by more than 2^8 many times); result vs the oracle.
+    V is a separate N(0,1) pool: with V aliasing the ramped K, |V| reaches ~16
+    and the bf16 rounding of P alone (2^-8 relative) exceeds the tolerance."""
+    lens = [1500, 700]
+    ps = 64
+    q, k, v, table, kl = _paged_inputs(lens, 128, 1, 576, ps, seed=37, Dv=512)
+    k = _ramp_keys(k, table, lens, ps, 3.0)
+    for S in (1, 2):
+        check_paged(q, k, v, table, kl, ps, scale, S, Dv=512, where=f"mla rescale scale={scale} S={S}")
+
+
+def test_mla_nan_past_kv_len_separate_v():
+    """Separate V pool, small pages (partial TMA box at the end), splits."""
+    lens = [90, 37]
+    ps = 16
+    q, k, v, table, kl = _paged_inputs(lens, 128, 1, 576, ps, seed=41, Dv=512)
+    kn, vn = k.clone(), v.clone()
+    for b, L in enumerate(lens):
+        last = table[b, (L - 1) // ps]
+        kn[last, :, L % ps:] = float("nan")
+        vn[last, :, L % ps:] = float("nan")
+    for S in (1, 3):
+        o1, l1 = paged_gpu(q, k, v, table, kl, ps, 0.04, S, o_dv=512)
+        o2, l2 = paged_gpu(q, kn, vn, table, kl, ps, 0.04, S, o_dv=512)
+        assert torch.isfinite(o2.float()).all()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_mla_paged_equals_contiguous_bitwise():
+    lens = [300, 64, 1000]
+    ps = 64
+    q, k, _, table, kl = _paged_inputs(lens, 128, 1, 576, ps, seed=43, alias=True)
+    o1, l1 = paged_gpu(q, k, k, table, kl, ps, 0.05, 1, o_dv=512)
+    n_pages = [(L + ps - 1) // ps for L in lens]
+    phys = np.concatenate([table[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
+    k2 = k[torch.as_tensor(phys, device=DEV)].contiguous()
+    t2 = np.full_like(table, -1)
+    pos = 0
+    for b, n in enumerate(n_pages):
+        t2[b, :n] = np.arange(pos, pos + n)
+        pos += n
+    o2, l2 = paged_gpu(q, k2, k2, t2, kl, ps, 0.05, 1, o_dv=512)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_mla_split_equals_unsplit():
+    lens = [5000, 129, 1]
+    q, k, _, table, kl = _paged_inputs(lens, 128, 1, 576, 64, seed=47, alias=True)
+    o1, l1 = paged_gpu(q, k, k, table, kl, 64, 0.05, 1, o_dv=512)
+    for S in (2, 7, 79):
+        o2, l2 = paged_gpu(q, k, k, table, kl, 64, 0.05, S, o_dv=512)
+        assert_o_close(o2, o1.float().cpu().numpy().astype(np.float64), f"mla split {S}")
+        assert np.max(np.abs(l2.cpu().numpy() - l1.cpu().numpy())) < 1e-4
+
+
 @pytest.mark.parametrize("Dv", [64, 128, 512])
 def test_split_merge_kernel_vs_oracle(Dv):
     S, R = 5, 300
