@@ -102,6 +102,26 @@ int encode_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
 }
 
+// 5D bf16 tensor map with 128-byte swizzle; strides in BYTES for dims 1..4.
+int encode_5d(CUtensorMap* map, const void* base, const uint64_t dims[5], const int64_t strides_b[4],
+              const uint32_t box[5]) {
+    cuuint64_t gdim[5], gstr[4];
+    cuuint32_t bdim[5], estr[5] = {1, 1, 1, 1, 1};
+    for (int i = 0; i < 5; ++i) {
+        if (dims[i] == 0 || dims[i] > (1ull << 32)) return ATTN_ERR_INVALID_ARG;
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+    }
+    for (int i = 0; i < 4; ++i) {
+        if (strides_b[i] <= 0 || (strides_b[i] % 16) != 0 || strides_b[i] >= (int64_t(1) << 40)) return ATTN_ERR_INVALID_ARG;
+        gstr[i] = (cuuint64_t)strides_b[i];
+    }
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), gdim, gstr, bdim,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -404,6 +424,8 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     const bool gqa = (Dqk == Dv && (Dqk == 64 || Dqk == 128) && G <= 16);
     if (!mla && !gqa) return ATTN_ERR_UNSUPPORTED;
     if (mla && Hkv != 1) return ATTN_ERR_UNSUPPORTED;
+    // MLA: a page box of min(page_size, 64) rows is the N of the score MMAs (16, 32 or 64)
+    if (mla && !(page_size % 64 == 0 || page_size == 32 || page_size == 16)) return ATTN_ERR_UNSUPPORTED;
     // a 64-key box is whole pages, or a page is whole boxes
     if (!(page_size % 64 == 0 || (64 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
@@ -430,7 +452,17 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     std::memset(&dp, 0, sizeof(dp));
     // rows per TMA box: one page, at most 64 keys
     const int box_rows = page_size < 64 ? page_size : 64;
-    {
+    if (mla) {
+        // (column in block, row in page, 64-column block, head, page); 3 blocks per K load, 4 per V load
+        const uint64_t dk[5] = {64, (uint64_t)page_size, 9, (uint64_t)Hkv, (uint64_t)num_pages};
+        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, k_pool_strides[2] * 2, k_pool_strides[0] * 2};
+        const uint32_t bk[5] = {64, (uint32_t)box_rows, (uint32_t)b2::MlaTcCfg::KB, 1, 1};
+        if (encode_5d(&dp.tm_k, k_pool, dk, sk, bk)) return ATTN_ERR_INVALID_ARG;
+        const uint64_t dv[5] = {64, (uint64_t)page_size, 8, (uint64_t)Hkv, (uint64_t)num_pages};
+        const int64_t sv[4] = {v_pool_strides[1] * 2, 128, v_pool_strides[2] * 2, v_pool_strides[0] * 2};
+        const uint32_t bv[5] = {64, (uint32_t)box_rows, (uint32_t)b2::MlaTcCfg::VB, 1, 1};
+        if (encode_5d(&dp.tm_v, v_pool, dv, sv, bv)) return ATTN_ERR_INVALID_ARG;
+    } else {
         const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
         const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
         const int64_t sk[3] = {k_pool_strides[1], k_pool_strides[2], k_pool_strides[0]};

@@ -128,11 +128,15 @@ __device__ __forceinline__ uint32_t peer_smem(uint32_t local, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void mbar_arrive_peer(uint32_t cluster_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+// Relaxed (no release ordering): for signals whose payload travels by bulk copy
+// (completed through the barrier's transaction count) or that only follow an
+// observed tensor-core completion.  A release at cluster scope here measured
+// 0.5-1.5 us per arrival on B200.
+__device__ __forceinline__ void mbar_arrive_peer_relaxed(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
-__device__ __forceinline__ void mbar_arrive_expect_tx_peer(uint32_t cluster_bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+__device__ __forceinline__ void mbar_arrive_expect_tx_peer_relaxed(uint32_t cluster_bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
                  "r"(bytes)
                  : "memory");
 }

@@ -119,6 +119,7 @@ def test_paged_rejects_bad_args_on_host(lib):
     assert call(Hkv=7) == rsd.ATTN_ERR_INVALID_ARG        # 64 % 7 != 0
     assert call(Hq=256, Hkv=8) == rsd.ATTN_ERR_UNSUPPORTED  # G = 32 > 16
     assert call(Dqk=576, Dv=512, Hq=128, Hkv=2) == rsd.ATTN_ERR_UNSUPPORTED  # MLA needs one KV head
+    assert call(Dqk=576, Dv=512, Hq=128, Hkv=1, ps=8) == rsd.ATTN_ERR_UNSUPPORTED  # MLA page box N >= 16
     assert call(splits=0) == rsd.ATTN_ERR_INVALID_ARG
 
 

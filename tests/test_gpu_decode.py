@@ -125,7 +125,7 @@ MLA_CASES = [
     ([500, 77], 128, 16, 1, False),
     ([600, 130], 128, 128, 3, True),
     ([3000], 16, 32, 5, True),
-    ([2, 64, 65], 128, 8, 2, False),
+    ([2, 64, 65, 200], 128, 16, 2, False),
 ]
 
 
