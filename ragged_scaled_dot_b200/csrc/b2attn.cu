@@ -394,13 +394,25 @@ int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_k
                               int num_sms) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_kv_len <= 0 || page_size <= 0 || num_sms <= 0) return 1;
     const bool mla = (Dqk == 576);
-    const int64_t ctas_per_split = mla ? (Hq / 64 > 0 ? Hq / 64 : 1) * (int64_t)B : (int64_t)Hkv * B;
-    const int64_t slots = (int64_t)num_sms * (mla ? 1 : 2);
-    int64_t s_balance = (8 * slots + ctas_per_split - 1) / ctas_per_split;
-    // keep the fp32 partials (written + read) under ~5% of the KV bytes streamed
+    int64_t s_balance;
+    double max_overhead;
+    if (mla) {
+        // a cluster of two CTAs (one per SM) per (sequence, split, 128-head group): about five
+        // waves of work units over the SM pairs, partial traffic up to ~10% of the KV bytes
+        const int64_t units_per_split = (int64_t)B * ((Hq + 127) / 128);
+        const int64_t pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
+        s_balance = (5 * pairs + units_per_split - 1) / units_per_split;
+        max_overhead = 0.10;
+    } else {
+        const int64_t ctas_per_split = (int64_t)Hkv * B;
+        const int64_t slots = (int64_t)num_sms * 2;
+        s_balance = (8 * slots + ctas_per_split - 1) / ctas_per_split;
+        max_overhead = 0.05;
+    }
+    // the fp32 partials (written + read) stay under max_overhead of the KV bytes streamed
     const double kv_bytes = 0.5 * (double)max_kv_len * Hkv * (double)(mla ? Dqk : Dqk + Dv) * 2.0;
     const double part_bytes_per_split = (double)Hq * Dv * 8.0;
-    int64_t s_traffic = (int64_t)(0.05 * kv_bytes / part_bytes_per_split);
+    int64_t s_traffic = (int64_t)(max_overhead * kv_bytes / part_bytes_per_split);
     int64_t s = s_balance < s_traffic ? s_balance : s_traffic;
     const int64_t max_pages = (max_kv_len + page_size - 1) / page_size;
     if (s > max_pages) s = max_pages;
