@@ -122,6 +122,16 @@ int encode_5d(CUtensorMap* map, const void* base, const uint64_t dims[5], const 
     return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
 }
 
+// Token-tile map for prefill: (column in block, token, 64-column block, head, batch),
+// strides in elements for token / head / batch; box = 128 tokens x all D/64 blocks.
+int encode_tok_tiles(CUtensorMap* map, const void* base, int D, int64_t H, int64_t T, int64_t Bn, int64_t ts,
+                     int64_t hs, int64_t bs) {
+    const uint64_t dims[5] = {64, (uint64_t)(T > 0 ? T : 1), (uint64_t)(D / 64), (uint64_t)H, (uint64_t)Bn};
+    const int64_t strides[4] = {ts * 2, 128, hs * 2, bs * 2};
+    const uint32_t box[5] = {64, 128, (uint32_t)(D / 64), 1, 1};
+    return encode_5d(map, base, dims, strides, box);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -235,17 +245,10 @@ int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* 
     const int D = Dqk;
     PrefillParams pp;
     std::memset(&pp, 0, sizeof(pp));
-    {
-        const uint32_t box[4] = {64, 1, 128, 1};
-        const uint64_t dq[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Sq, (uint64_t)B};
-        const int64_t sq[3] = {q_strides[2], q_strides[1], q_strides[0]};
-        if (encode_4d(&pp.tm_q, q, dq, sq, box)) return ATTN_ERR_INVALID_ARG;
-        const uint64_t dkv[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)(Skv > 0 ? Skv : 1), (uint64_t)B};
-        const int64_t sk[3] = {k_strides[2], k_strides[1], k_strides[0]};
-        const int64_t sv[3] = {v_strides[2], v_strides[1], v_strides[0]};
-        if (encode_4d(&pp.tm_k, k, dkv, sk, box)) return ATTN_ERR_INVALID_ARG;
-        if (encode_4d(&pp.tm_v, v, dkv, sv, box)) return ATTN_ERR_INVALID_ARG;
-    }
+    if (encode_tok_tiles(&pp.tm_q, q, D, Hq, Sq, B, q_strides[1], q_strides[2], q_strides[0]) ||
+        encode_tok_tiles(&pp.tm_k, k, D, Hkv, Skv, B, k_strides[1], k_strides[2], k_strides[0]) ||
+        encode_tok_tiles(&pp.tm_v, v, D, Hkv, Skv, B, v_strides[1], v_strides[2], v_strides[0]))
+        return ATTN_ERR_INVALID_ARG;
     int hpi, n_pairs;
     pair_shape(Hq, Hkv, &hpi, &n_pairs);
     pp.mode = 0;
@@ -309,17 +312,13 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
 
     PrefillParams pp;
     std::memset(&pp, 0, sizeof(pp));
-    {
-        const uint32_t box[4] = {64, 1, 128, 1};
-        const uint64_t dq[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)total_q, 1};
-        const int64_t sq[3] = {q_strides[1], q_strides[0], unit_dim_stride(q_strides[0] * total_q, 8)};
-        if (encode_4d(&pp.tm_q, q, dq, sq, box)) return ATTN_ERR_INVALID_ARG;
-        const uint64_t dkv[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)(total_kv > 0 ? total_kv : 1), 1};
-        const int64_t sk[3] = {k_strides[1], k_strides[0], unit_dim_stride(k_strides[0] * total_kv, 8)};
-        const int64_t sv[3] = {v_strides[1], v_strides[0], unit_dim_stride(v_strides[0] * total_kv, 8)};
-        if (encode_4d(&pp.tm_k, k, dkv, sk, box)) return ATTN_ERR_INVALID_ARG;
-        if (encode_4d(&pp.tm_v, v, dkv, sv, box)) return ATTN_ERR_INVALID_ARG;
-    }
+    if (encode_tok_tiles(&pp.tm_q, q, D, Hq, total_q, 1, q_strides[0], q_strides[1],
+                         unit_dim_stride(q_strides[0] * total_q, 8)) ||
+        encode_tok_tiles(&pp.tm_k, k, D, Hkv, total_kv, 1, k_strides[0], k_strides[1],
+                         unit_dim_stride(k_strides[0] * total_kv, 8)) ||
+        encode_tok_tiles(&pp.tm_v, v, D, Hkv, total_kv, 1, v_strides[0], v_strides[1],
+                         unit_dim_stride(v_strides[0] * total_kv, 8)))
+        return ATTN_ERR_INVALID_ARG;
     int hpi, n_pairs;
     pair_shape(Hq, Hkv, &hpi, &n_pairs);
     const int G = Hq / Hkv;

@@ -89,15 +89,6 @@ static_assert(MlaTcCfg::SMEM <= 232448, "shared memory");
 static_assert(MlaTcCfg::RK <= 8 && MlaTcCfg::RV <= 8, "barrier area");
 static_assert(9 % MlaTcCfg::KB == 0 && 8 % MlaTcCfg::VB == 0 && MlaTcCfg::VB % 2 == 0 && MlaTcCfg::VLOADS <= 2, "blocks");
 
-__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
-                                            int c2, int c3, int c4) {
-    asm volatile(
-        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
-        : "memory");
-}
-
 // Page ids of the np = 64 / R page boxes of the chunk starting at key t0.  The
 // loads are only issued here; the producer fetches the next chunk's ids while
 // it issues the current chunk's boxes.  Bit i of the result: box i holds keys

@@ -47,7 +47,8 @@
 namespace b2 {
 
 struct PrefillParams {
-    CUtensorMap tm_q;  // 4D (d, head, token, batch), 128B swizzle, box (64, 1, 128, 1)
+    CUtensorMap tm_q;  // 5D (d in block, token, 64-column block, head, batch), 128B swizzle,
+                       // box (64, 128, D/64, 1, 1): one request per tile reads whole rows
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     int mode;  // 0 dense, 1 ragged
@@ -231,9 +232,7 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
             if (!mbar_wait(b_qempty, (q_it & 1) ^ 1, abort_flag)) { ok = false; break; }
             mbar_arrive_expect_tx(b_qfull, it.nh * TILE);
             for (int s = 0; s < it.nh; ++s)
-                for (int hf = 0; hf < C::HALVES; ++hf)
-                    tma_load_4d(sQ + s * TILE + hf * 16384u, &p.tm_q, b_qfull, hf * 64, it.h0 + s,
-                                it.q_tok0, it.batch);
+                tma_load_5d(sQ + s * TILE, &p.tm_q, b_qfull, 0, it.q_tok0, 0, it.h0 + s, it.batch);
             ++q_it;
             const int g = it.h0 / p.G;
             for (int j = 0; ok && j < it.n_kv; ++j) {
@@ -242,9 +241,7 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
                     if (!mbar_wait(empty_bar(st), ((kv_it / NST) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar(st), TILE);
                     const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
-                    for (int hf = 0; hf < C::HALVES; ++hf)
-                        tma_load_4d(sKV + st * TILE + hf * 16384u, map, full_bar(st), hf * 64, g,
-                                    it.kv_tok0 + j * 128, it.batch);
+                    tma_load_5d(sKV + st * TILE, map, full_bar(st), 0, it.kv_tok0 + j * 128, 0, g, it.batch);
                     ++kv_it;
                 }
             }
