@@ -180,6 +180,10 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  *   Absorbed MLA: pass v_pool == k_pool with Dv < Dqk; V is then the first Dv
  *   columns of each K row ("cuDNN Frontend v1.32.0 Release Notes", "SDPA:
  *   wider native forward support": Q/K576, V512, absorbed-MLA cache layouts).
+ *   MLA (Dqk 576, Dv 512) needs Hkv == 1 and page_size 16, 32 or a multiple
+ *   of 64 (ATTN_ERR_UNSUPPORTED otherwise); any Hq (groups of 128 heads).
+ *   GQA needs page_size dividing or divisible by 64 (at least 8) and
+ *   Hq / Hkv <= 16.
  *   Each page-table row holds at least ceil(max_kv_len / page_size) entries.
  *   kv_lens: DEVICE int32 [B], each in [0, max_kv_len]; page ids must lie in
  *   [0, num_pages).  Violations set ATTN_ERR_DEVICE_INPUT on the device.
