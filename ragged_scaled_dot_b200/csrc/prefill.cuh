@@ -130,7 +130,8 @@ struct PrefillCfg {
     static constexpr int NST = (D == 128) ? 5 : 8;     // K/V ring depth
     static constexpr int NRING = 2;                    // published work items in flight
     static constexpr uint32_t BAR_OFF = (2 + NST) * TILE;
-    static constexpr uint32_t SMEM = BAR_OFF + 256 + 1024;  // + barriers + alignment slack
+    // + barriers, tmem address, abort flag, item ring (up to 264 bytes at D = 64) + alignment slack
+    static constexpr uint32_t SMEM = BAR_OFF + 512 + 1024;
 };
 
 // Exponentials per 32-column chunk evaluated on the FMA pipe (the rest on MUFU).
