@@ -266,6 +266,22 @@ def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
     return Part(name, "GB/s", nbytes / 1e9, launches, step, e2e_setup, info), data
 
 
+def rank_seed_offset(rank):
+    """Each rank draws its own synthetic batch of the same shape (weak scaling)."""
+    return 1000 * rank
+
+
+def reduce_over_ranks(value, dist, op, device):
+    """One number reduced over all ranks (MAX for times, SUM for units of work);
+    the value itself on a single process.  Every rank must call it in the same order."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
 def time_part(torch, part, steps, warmup, dist, world):
     """Device time of `steps` back-to-back steps (barrier + sync on both sides),
     max over ranks; also per-step event durations on the launching stream."""
@@ -285,9 +301,7 @@ def time_part(torch, part, steps, warmup, dist, world):
     total_ms = ev[0].elapsed_time(ev[-1])
     per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
     if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+        total_ms = reduce_over_ranks(total_ms, dist, dist.ReduceOp.MAX, "cuda")
         dist.barrier()
     return total_ms, per
 
@@ -308,9 +322,7 @@ def time_e2e(torch, part, steps, dist):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = reduce_over_ranks(ms, dist, dist.ReduceOp.MAX, "cuda")
     return ms, h2d, d2h
 
 
@@ -403,12 +415,13 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     num_sms = torch.cuda.get_device_properties(local).multi_processor_count
 
-    prefill, pdata = make_ragged_prefill(torch, rsd, synth, dev, rank * 1000)
-    decode, ddata = make_paged(torch, rsd, synth, dev, rank * 1000, "paged_decode", num_sms)
+    off = rank_seed_offset(rank)
+    prefill, pdata = make_ragged_prefill(torch, rsd, synth, dev, off)
+    decode, ddata = make_paged(torch, rsd, synth, dev, off, "paged_decode", num_sms)
     extras = []
     if not args.no_extras:
-        extras.append(make_dense_prefill(torch, rsd, synth, dev, rank * 1000)[0])
-        mla, _ = make_paged(torch, rsd, synth, dev, rank * 1000, "mla_decode", num_sms)
+        extras.append(make_dense_prefill(torch, rsd, synth, dev, off)[0])
+        mla, _ = make_paged(torch, rsd, synth, dev, off, "mla_decode", num_sms)
         extras.append(mla)
     torch.cuda.synchronize()
 
@@ -419,10 +432,14 @@ def run_ours(args):
             results[part.name] = (total_ms, per)
     assert rsd.attn_get_device_error() == rsd.ATTN_OK, "device-side error during the bench"
 
+    sum_op = dist.ReduceOp.SUM if dist is not None else None
+    # units of work of all ranks (their seeded batches differ in length)
+    all_units = {p.name: reduce_over_ranks(p.units, dist, sum_op, "cuda") for p in [prefill, decode] + extras}
+
     def part_summary(part, bound):
         total_ms, per = results[part.name]
         ms = total_ms / args.steps
-        value = part.units * world / (total_ms / 1e3 / args.steps)
+        value = all_units[part.name] / (total_ms / 1e3 / args.steps)
         # dominant kernel: the part's launch sequence, timed per step on its stream
         kern_ms = statistics.mean(per)
         if bound == "tensor":
@@ -452,7 +469,7 @@ def run_ours(args):
     e2e = {}
     for part in ((prefill, decode) if not args.no_e2e else ()):
         ms, h2d, d2h = time_e2e(torch, part, max(1, min(3, args.steps)), dist)
-        e2e[part.name] = {"value": round(part.units * world / (ms / 1e3 / max(1, min(3, args.steps))), 3),
+        e2e[part.name] = {"value": round(all_units[part.name] / (ms / 1e3 / max(1, min(3, args.steps))), 3),
                           "unit": part.unit, "h2d_bytes_per_step": int(h2d),
                           "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / max(1, min(3, args.steps)), 3)}
 
