@@ -200,9 +200,9 @@ int noalloc_scratch(void** out) {
 int launch_prefill(PrefillParams& pp, int D, int grid, cudaStream_t st) {
     if (grid <= 0) return ATTN_OK;
     if (D == 128)
-        b2::prefill_kernel<128><<<grid, 384, b2::PrefillCfg<128>::SMEM, st>>>(pp);
+        b2::prefill_kernel<128><<<grid, 320, b2::PrefillCfg<128>::SMEM, st>>>(pp);
     else
-        b2::prefill_kernel<64><<<grid, 384, b2::PrefillCfg<64>::SMEM, st>>>(pp);
+        b2::prefill_kernel<64><<<grid, 320, b2::PrefillCfg<64>::SMEM, st>>>(pp);
     return launch_status();
 }
 

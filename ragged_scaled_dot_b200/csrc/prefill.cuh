@@ -9,7 +9,7 @@
 // pair), so the CTAs working at the same time share one sequence-head's K/V
 // in L2 and the long items start first.
 //
-// Warp roles (384 threads):
+// Warp roles (320 threads):
 //   warp 0      claims items, publishes them to the other roles through a
 //               small shared-memory ring, and issues the TMA loads: Q tiles of
 //               the item, then K(j), V(j) into a ring of NST stages.
@@ -17,8 +17,11 @@
 //               (descriptor bases are precomputed: this thread shares its SM
 //               sub-partition with two busy softmax warps, so every instruction
 //               it issues is expensive).
-//   warps 4-7   softmax for slot 0 (query head h0), one TMEM lane (row) each.
-//   warps 8-11  softmax for slot 1 (query head h0 + 1).
+//   warps 2-5   softmax for slot 0 (query head h0), one TMEM lane (row) each:
+//               any four consecutive warps cover the four TMEM lane quadrants.
+//   warps 6-9   softmax for slot 1 (query head h0 + 1).
+// Ten warps (not twelve) leave each thread about 200 registers, enough for a
+// 128-column score row without spilling.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
 // P (bf16) overwrites the first 64 columns of its S tile and feeds the PV MMA
 // straight from TMEM.
@@ -138,7 +141,7 @@ struct PrefillCfg {
 constexpr int kEmuPer32 = 0;
 
 template <int D>
-__global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
+__global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     using C = PrefillCfg<D>;
     constexpr int NST = C::NST;
     constexpr int NRING = C::NRING;
@@ -338,9 +341,9 @@ __global__ void __launch_bounds__(384, 1) prefill_kernel(const __grid_constant__
         // Wait for every MMA this thread issued before TMEM is released.
         tc_commit(b_drain);
         mbar_wait(b_drain, 0, nullptr, 100000000ull);
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         // ------------------------------------------------------------ softmax
-        const int slot = (warp - 4) >> 2;
+        const int slot = (warp - 2) >> 2;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
