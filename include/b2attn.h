@@ -202,6 +202,39 @@ int attn_fwd_paged(const void *q, const void *k_pool, const void *v_pool, void *
                    float scale, int num_splits,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Ragged queries over a paged K/V cache: chunked prefill and multi-token
+ * decode ("cuDNN Frontend v1.31.0 Release Notes", "SDPA: paged KV, split-KV,
+ * and engine selection": paged K/V for prefill; "cuDNN Frontend v1.28.0
+ * release notes", ragged / THD queries).  Sequence b has
+ * Lq_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] queries, the LAST Lq_b positions
+ * of its kv_lens[b] cached keys: with causal, query i sees keys
+ * j <= i + kv_lens[b] - Lq_b (bottom-right); Lq_b > kv_lens[b] leaves the
+ * first rows without keys (O = 0, LSE = -inf).
+ *   q, o: packed THD [total_q, Hq, D], (token, head) element strides.
+ *   k_pool / v_pool, page_table, kv_lens: as for attn_fwd_paged (DEVICE).
+ *   lse / lse_layout: as for attn_fwd_ragged.
+ * Supported: D = Dqk = Dv in {64, 128}, Hq % Hkv == 0, page_size dividing 128
+ * (at least 8) or a multiple of 128, and pools whose page stride is a whole
+ * number of 8-row groups (page stride % (8 * row stride) == 0, the same for K
+ * and V; dense HND and NHD pools qualify); else ATTN_ERR_UNSUPPORTED.
+ * workspace: >= attn_fwd_paged_prefill_workspace_size(...) bytes, 256-byte
+ * aligned.  Row slots past kv_len inside a sequence's last page are never
+ * read into O (stale or NaN values are zeroed on chip).
+ */
+int attn_fwd_paged_prefill(const void *q, const void *k_pool, const void *v_pool, void *o,
+                           float *lse, const int32_t *cu_seqlens_q, const int32_t *page_table,
+                           int64_t page_table_stride, const int32_t *kv_lens, int B,
+                           int max_seqlen_q, int64_t total_q, int Hq, int Hkv, int D,
+                           int page_size, int64_t num_pages, int max_kv_len,
+                           const int64_t q_strides[2], const int64_t o_strides[2],
+                           const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
+                           int lse_layout, float scale, int causal,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes attn_fwd_paged_prefill needs (the work list of attn_fwd_ragged). */
+size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv);
+
 /* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1). */
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits);
 

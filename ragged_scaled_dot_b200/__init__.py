@@ -45,6 +45,9 @@ SIGNATURES = {
     "attn_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _I, _I, _I, _I, _L, _I,
                             _L2, _L2, _L3, _L3, _F, _I, _P, _Z, _P]),
     "attn_fwd_paged_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "attn_fwd_paged_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _L, _I, _I, _I, _I, _L, _I,
+                                    _L2, _L2, _L3, _L3, _I, _F, _I, _P, _Z, _P]),
+    "attn_fwd_paged_prefill_workspace_size": (_Z, [_I, _I, _L, _I, _I]),
     "attn_paged_suggest_splits": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "attn_split_merge": (_I, [_P, _P, _I, _L, _I, _P, _L, _P, _P]),
     "attn_get_device_error": (_I, [_P]),
@@ -213,6 +216,36 @@ def attn_fwd_paged(q, k_pool, v_pool, o, lse, page_table, kv_lens, *, page_size:
         _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout),
         pool_strides(v_pool, kv_layout), float(scale), int(num_splits), _ptr(workspace),
         ws_bytes, _stream(stream)), "attn_fwd_paged")
+
+
+def attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv) -> int:
+    return int(lib().attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv))
+
+
+def attn_fwd_paged_prefill(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, kv_lens, *,
+                           max_seqlen_q: int, page_size: int, max_kv_len: int, scale: float,
+                           causal: bool, workspace, lse_layout: int = ATTN_LSE_PADDED_BSH,
+                           kv_layout: str = "HND", total_q=None, stream=None):
+    """Ragged queries over a paged cache (chunked prefill, multi-token decode):
+    q [T,Hq,D] packed by cu_seqlens_q (int32 CUDA [B+1]); sequence b's queries are
+    the last Lq_b positions of its kv_lens[b] keys (bottom-right causal).  Pools 4D
+    in kv_layout, page_table int32 CUDA [B,max_pages], o [T,Hq,D], lse as in
+    attn_fwd_ragged.  workspace: uint8 CUDA tensor."""
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (o, "o")):
+        _bf16(t, n)
+    B = cu_seqlens_q.numel() - 1
+    Hq, D = q.shape[1], q.shape[2]
+    Hkv = k_pool.shape[1] if kv_layout == "HND" else k_pool.shape[2]
+    num_pages = k_pool.shape[0]
+    total_q = q.shape[0] if total_q is None else total_q
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().attn_fwd_paged_prefill(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(page_table),
+        int(page_table.stride(0)), _ptr(kv_lens), B, int(max_seqlen_q), int(total_q), Hq, Hkv, D,
+        int(page_size), int(num_pages), int(max_kv_len), _L2(q.stride(0), q.stride(1)),
+        _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout), pool_strides(v_pool, kv_layout),
+        int(lse_layout), float(scale), int(causal), _ptr(workspace), ws_bytes, _stream(stream)),
+        "attn_fwd_paged_prefill")
 
 
 # --------------------------------------------------------------------- merge

@@ -22,17 +22,24 @@ namespace b2 {
 // ---------------------------------------------------------------------------
 constexpr int kSortBuckets = 4096;
 
-__device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t* cu_kv, int b,
-                                              int max_sq, int max_skv, int64_t total_q,
+// Key lengths come from cu_kv (ragged K/V) or, when kv_lens is given, from
+// kv_lens (K/V in a paged cache).
+__device__ __forceinline__ int seq_kv_len(const int32_t* cu_kv, const int32_t* kv_lens, int b) {
+    return kv_lens ? kv_lens[b] : cu_kv[b + 1] - cu_kv[b];
+}
+
+__device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t* cu_kv, const int32_t* kv_lens,
+                                              int b, int max_sq, int max_skv, int64_t total_q,
                                               int64_t total_kv) {
-    const int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_kv[b], k1 = cu_kv[b + 1];
-    const int lq = q1 - q0, lk = k1 - k0;
-    return q0 >= 0 && k0 >= 0 && lq >= 0 && lk >= 0 && lq <= max_sq && lk <= max_skv &&
-           (int64_t)q1 <= total_q && (int64_t)k1 <= total_kv;
+    const int q0 = cu_q[b], q1 = cu_q[b + 1];
+    const int lq = q1 - q0, lk = seq_kv_len(cu_kv, kv_lens, b);
+    const bool kv_ok = kv_lens ? true : (cu_kv[b] >= 0 && (int64_t)cu_kv[b + 1] <= total_kv);
+    return q0 >= 0 && kv_ok && lq >= 0 && lk >= 0 && lq <= max_sq && lk <= max_skv && (int64_t)q1 <= total_q;
 }
 
 __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
-    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv, int B, int max_sq,
+    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv,
+    const int32_t* __restrict__ kv_lens, int B, int max_sq,
     int max_skv, int64_t total_q, int64_t total_kv, int causal, int Hkv, int pairs_per_group,
     int heads_per_item, int G, int* __restrict__ header, int4* __restrict__ items,
     int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles) {
@@ -43,13 +50,13 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     for (int i = tid; i < kSortBuckets; i += blockDim.x) hist[i] = 0;
     if (tid == 0) {
         n_tiles_sh = 0;
-        if (cu_q[0] != 0 || cu_kv[0] != 0) record_status(ATTN_ERR_DEVICE_INPUT);
+        if (cu_q[0] != 0 || (kv_lens == nullptr && cu_kv[0] != 0)) record_status(ATTN_ERR_DEVICE_INPUT);
     }
     __syncthreads();
     // 1. validate, histogram of query-tile counts
     for (int b = tid; b < B; b += blockDim.x) {
         int nqt = 0;
-        if (ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv))
+        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv))
             nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
         else
             record_status(ATTN_ERR_DEVICE_INPUT);
@@ -69,7 +76,7 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) {
         int nqt = 0;
-        if (ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv))
+        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv))
             nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
         const int r = atomicAdd(&hist[min(nqt, kSortBuckets - 1)], 1);
         rank_of[b] = r;
@@ -117,8 +124,8 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     // 3. items of each sequence: (kv head, query tile longest first, head pair)
     const int n_pairs = Hkv * pairs_per_group;
     for (int b = tid; b < B; b += blockDim.x) {
-        if (!ragged_seq_ok(cu_q, cu_kv, b, max_sq, max_skv, total_q, total_kv)) continue;
-        const int lq = cu_q[b + 1] - cu_q[b], lk = cu_kv[b + 1] - cu_kv[b];
+        if (!ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) continue;
+        const int lq = cu_q[b + 1] - cu_q[b], lk = seq_kv_len(cu_kv, kv_lens, b);
         const int nqt = (lq + 127) >> 7;
         const int tile0 = sorted_nqt[rank_of[b]];  // first tile slot of this sequence
         if (tile0 + nqt > max_tiles) continue;

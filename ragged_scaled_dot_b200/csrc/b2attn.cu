@@ -57,10 +57,16 @@ int setup_device(int* dev_out, int* sms_out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return ATTN_ERR_CUDA;
         cudaError_t e = cudaSuccess;
-        e = cudaFuncSetAttribute(b2::prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(b2::prefill_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  b2::PrefillCfg<64>::SMEM);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(b2::prefill_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(b2::prefill_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::PrefillCfg<128>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::prefill_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     b2::PrefillCfg<64>::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(b2::prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::PrefillCfg<128>::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(b2::decode_gqa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -199,10 +205,18 @@ int noalloc_scratch(void** out) {
 // Launches the prefill kernel for an already-filled PrefillParams.
 int launch_prefill(PrefillParams& pp, int D, int grid, cudaStream_t st) {
     if (grid <= 0) return ATTN_OK;
-    if (D == 128)
-        b2::prefill_kernel<128><<<grid, 320, b2::PrefillCfg<128>::SMEM, st>>>(pp);
-    else
-        b2::prefill_kernel<64><<<grid, 320, b2::PrefillCfg<64>::SMEM, st>>>(pp);
+    const bool paged = (pp.mode == 2);
+    if (D == 128) {
+        if (paged)
+            b2::prefill_kernel<128, true><<<grid, 320, b2::PrefillCfg<128>::SMEM, st>>>(pp);
+        else
+            b2::prefill_kernel<128, false><<<grid, 320, b2::PrefillCfg<128>::SMEM, st>>>(pp);
+    } else {
+        if (paged)
+            b2::prefill_kernel<64, true><<<grid, 320, b2::PrefillCfg<64>::SMEM, st>>>(pp);
+        else
+            b2::prefill_kernel<64, false><<<grid, 320, b2::PrefillCfg<64>::SMEM, st>>>(pp);
+    }
     return launch_status();
 }
 
@@ -329,7 +343,7 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     int4* items = reinterpret_cast<int4*>(wsb + wl.items_off);
 
     b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
-        cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv, total_q, total_kv, causal, Hkv, G / hpi,
+        cu_seqlens_q, cu_seqlens_kv, nullptr, B, max_seqlen_q, max_seqlen_kv, total_q, total_kv, causal, Hkv, G / hpi,
         hpi, G, header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
         max_tiles);
     if (int e = launch_status()) return e;
@@ -381,6 +395,118 @@ int attn_fwd_ragged_noalloc(const void* q, const void* k, const void* v, void* o
 }
 
 size_t attn_fwd_ragged_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+// ------------------------------------------------ paged prefill (chunked)
+size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv) {
+    return attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
+}
+
+int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
+                           const int32_t* cu_seqlens_q, const int32_t* page_table, int64_t page_table_stride,
+                           const int32_t* kv_lens, int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv,
+                           int D, int page_size, int64_t num_pages, int max_kv_len, const int64_t q_strides[2],
+                           const int64_t o_strides[2], const int64_t k_pool_strides[3],
+                           const int64_t v_pool_strides[3], int lse_layout, float scale, int causal,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (B < 0 || max_seqlen_q < 0 || total_q < 0 || max_kv_len < 0 || num_pages < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+    if (lse_layout != ATTN_LSE_PADDED_BSH && lse_layout != ATTN_LSE_PACKED_TH) return ATTN_ERR_INVALID_ARG;
+    if (!q_strides || !o_strides || !k_pool_strides || !v_pool_strides) return ATTN_ERR_INVALID_ARG;
+    if (page_size <= 0 || page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    // a page box of min(page_size, 128) rows: whole 8-row groups that tile a 128-key tile
+    if (!(page_size % 128 == 0 || (128 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
+    if (total_q >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+    if (!q || !k_pool || !v_pool || !o || !cu_seqlens_q || !page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (num_pages == 0) return ATTN_ERR_INVALID_ARG;
+    if (B > 1 && page_table_stride < ((int64_t)max_kv_len + page_size - 1) / page_size) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 2; ++i)
+        if (!stride_ok(q_strides[i]) || !stride_ok(o_strides[i])) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (!stride_ok(k_pool_strides[i]) || !stride_ok(v_pool_strides[i])) return ATTN_ERR_INVALID_ARG;
+    // the maps address a page as whole 8-row groups: page stride = groups_per_page x 8 rows,
+    // the same for K and V
+    const int64_t gk = k_pool_strides[0] / (8 * k_pool_strides[1]);
+    const int64_t gv = v_pool_strides[0] / (8 * v_pool_strides[1]);
+    if (k_pool_strides[0] % (8 * k_pool_strides[1]) != 0 || v_pool_strides[0] % (8 * v_pool_strides[1]) != 0 ||
+        gk != gv || gk < page_size / 8)
+        return ATTN_ERR_UNSUPPORTED;
+    if ((int64_t)num_pages * gk >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
+    const size_t need = attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
+    if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
+    int dev, sms;
+    if (int e = setup_device(&dev, &sms)) return e;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int R = page_size < 128 ? page_size : 128;
+
+    PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    if (encode_tok_tiles(&pp.tm_q, q, D, Hq, total_q, 1, q_strides[0], q_strides[1],
+                         unit_dim_stride(q_strides[0] * total_q, 8)))
+        return ATTN_ERR_INVALID_ARG;
+    {
+        // (column in block, row in 8-row group, 64-column block, 8-row group of the pool, head)
+        const uint64_t dims[5] = {64, 8, (uint64_t)(D / 64), (uint64_t)(num_pages * gk), (uint64_t)Hkv};
+        const uint32_t box[5] = {64, 8, (uint32_t)(D / 64), (uint32_t)(R / 8), 1};
+        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, 8 * k_pool_strides[1] * 2, k_pool_strides[2] * 2};
+        const int64_t sv[4] = {v_pool_strides[1] * 2, 128, 8 * v_pool_strides[1] * 2, v_pool_strides[2] * 2};
+        if (encode_5d(&pp.tm_k, k_pool, dims, sk, box) || encode_5d(&pp.tm_v, v_pool, dims, sv, box))
+            return ATTN_ERR_INVALID_ARG;
+    }
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int G = Hq / Hkv;
+    const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
+    const RaggedWs wl = ragged_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv);
+    char* wsb = static_cast<char*>(workspace);
+    int* header = reinterpret_cast<int*>(wsb);
+    int4* items = reinterpret_cast<int4*>(wsb + wl.items_off);
+    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
+        cu_seqlens_q, nullptr, kv_lens, B, max_seqlen_q, max_kv_len, total_q, 0, causal, Hkv, G / hpi, hpi, G,
+        header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
+        max_tiles);
+    if (int e = launch_status()) return e;
+    if (lse != nullptr && lse_layout == ATTN_LSE_PADDED_BSH) {
+        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
+        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
+        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
+        if (int e = launch_status()) return e;
+    }
+    pp.mode = 2;
+    pp.B = B;
+    pp.Hq = Hq;
+    pp.Hkv = Hkv;
+    pp.G = G;
+    pp.heads_per_item = hpi;
+    pp.pairs_per_group = G / hpi;
+    pp.cu_q = cu_seqlens_q;
+    pp.items = items;
+    pp.header = header;
+    pp.o = static_cast<__nv_bfloat16*>(o);
+    pp.o_ts = o_strides[0];
+    pp.o_hs = o_strides[1];
+    pp.lse = lse;
+    pp.lse_layout = (lse_layout == ATTN_LSE_PADDED_BSH) ? 1 : 2;
+    pp.lse_smax = max_seqlen_q;
+    pp.scale_log2 = scale * kLog2e;
+    pp.causal = causal;
+    pp.kv_lens = kv_lens;
+    pp.page_table = page_table;
+    pp.pt_stride = page_table_stride;
+    pp.page_size = page_size;
+    pp.box_rows = R;
+    pp.num_pages = num_pages;
+    pp.groups_per_page = (int)gk;
+    pp.n_groups = (int)(num_pages * gk);
+    pp.max_kv_len = max_kv_len;
+    const int64_t items_max = (int64_t)max_tiles * n_pairs;
+    const int grid = (int)(items_max < sms ? items_max : sms);
+    return launch_prefill(pp, D, grid, st);
+}
 
 // ------------------------------------------------------------------ paged
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits) {

@@ -72,6 +72,17 @@ struct PrefillParams {
     int lse_smax;
     float scale_log2;
     int causal;
+    // mode 2 (queries of a ragged batch over a paged K/V cache): key t of
+    // sequence b is row t % page_size of page page_table[b * pt_stride + t / page_size];
+    // the pool maps address 8-row groups: group = page * groups_per_page + row / 8
+    const int32_t* kv_lens;
+    const int32_t* page_table;
+    int64_t pt_stride;
+    int page_size, box_rows;  // box_rows = min(page_size, 128) rows per page box
+    int64_t num_pages;
+    int groups_per_page;      // page stride / (8 x row stride) of the pool
+    int n_groups;             // extent of the pool maps' group dimension (the zero-fill coordinate)
+    int max_kv_len;
 };
 
 struct PrefillItem {
@@ -115,15 +126,48 @@ __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx
         it.qt = w.y;
         it.h0 = w.z;
         const int q0 = __ldg(p.cu_q + it.b), q1 = __ldg(p.cu_q + it.b + 1);
-        const int k0 = __ldg(p.cu_kv + it.b), k1 = __ldg(p.cu_kv + it.b + 1);
         it.Lq = q1 - q0;
-        it.Lkv = k1 - k0;
         it.q_tok0 = q0 + it.qt * 128;
-        it.kv_tok0 = k0;
         it.batch = 0;
+        if (p.mode == 2) {
+            // validated by the work-list kernel: items exist only for sequences with 0 <= kv_len <= max
+            it.Lkv = __ldg(p.kv_lens + it.b);
+            it.kv_tok0 = 0;
+        } else {
+            const int k0 = __ldg(p.cu_kv + it.b), k1 = __ldg(p.cu_kv + it.b + 1);
+            it.Lkv = k1 - k0;
+            it.kv_tok0 = k0;
+        }
     }
     it.nh = p.heads_per_item;
     it.n_kv = prefill_n_kv(it.qt, it.Lq, it.Lkv, p.causal);
+}
+
+// Mode 2 K/V tile of 128 keys from t0: 128 / box_rows page boxes, each
+// (64 columns, 8 rows, D/64 blocks, box_rows/8 groups, 1 head) landing as
+// [group][block][8 rows][128 B].  Two 64-row boxes placed back to back keep
+// one uniform 8-row-group stride, so the tile is a single MMA operand across
+// pages.  Boxes at or past Lkv (or with a bad page id, recorded) read zeros.
+__device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const CUtensorMap* map, uint32_t dst,
+                                                 uint32_t bar, int b, int g, int t0, int Lkv, uint32_t box_bytes) {
+    for (int i = 0; i < 128 / p.box_rows; ++i) {
+        const int t = t0 + i * p.box_rows;
+        int gg = p.n_groups;
+        if (t < Lkv) {
+            const int page = __ldg(p.page_table + (int64_t)b * p.pt_stride + t / p.page_size);
+            if (page < 0 || (int64_t)page >= p.num_pages)
+                record_status(ATTN_ERR_DEVICE_INPUT);
+            else
+                gg = page * p.groups_per_page + (t % p.page_size) / 8;
+        }
+        tma_load_5d(dst + (uint32_t)i * box_bytes, map, bar, 0, 0, 0, gg, g);
+    }
+}
+
+// Mode 2: does the K/V tile from t0 end inside a page box that runs past Lkv
+// (rows past the sequence that can hold stale values, possibly NaN)?
+__device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int t0, int Lkv) {
+    return t0 < Lkv && Lkv <= t0 + 128 && (Lkv % p.box_rows) != 0;
 }
 
 template <int D>
@@ -140,7 +184,7 @@ struct PrefillCfg {
 // Exponentials per 32-column chunk evaluated on the FMA pipe (the rest on MUFU).
 constexpr int kEmuPer32 = 0;
 
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
     using C = PrefillCfg<D>;
     constexpr int NST = C::NST;
@@ -167,7 +211,8 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
     const uint32_t b_drain = b_qfull + 80;
     const uint32_t b_ifull0 = b_qfull + 88;              // + 8*ring slot
     const uint32_t b_iempty0 = b_ifull0 + 8 * NRING;     // + 8*ring slot
-    const uint32_t misc = 16u * NST + 88 + 16 * NRING;   // byte offset past the barriers
+    const uint32_t b_vtail0 = b_iempty0 + 8 * NRING;     // + 8*stage: tail rows of a V tile zeroed
+    const uint32_t misc = 16u * NST + 88 + 16 * NRING + 8 * NST;  // byte offset past the barriers
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(sgen + C::BAR_OFF + misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + misc + 4);
     volatile int* item_ring = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + misc + 8);
@@ -189,6 +234,7 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
             mbar_init(b_oempty0 + 8 * s, 128);
         }
         mbar_init(b_drain, 1);
+        for (int i = 0; i < NST; ++i) mbar_init(b_vtail0 + 8 * i, 1);
         for (int r = 0; r < NRING; ++r) {
             mbar_init(b_ifull0 + 8 * r, 1);
             mbar_init(b_iempty0 + 8 * r, 9);  // MMA thread + one lane of each softmax warp
@@ -245,7 +291,26 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     if (!mbar_wait(empty_bar(st), ((kv_it / NST) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar(st), TILE);
                     const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
-                    tma_load_5d(sKV + st * TILE, map, full_bar(st), 0, it.kv_tok0 + j * 128, 0, g, it.batch);
+                    if constexpr (PAGED) {
+                        const uint32_t box_bytes = (uint32_t)p.box_rows * (D / 64) * 128u;
+                        paged_issue_tile(p, map, sKV + st * TILE, full_bar(st), it.b, g, j * 128, it.Lkv, box_bytes);
+                        if (t == 1 && paged_tile_has_tail(p, j * 128, it.Lkv)) {
+                            // value rows past the sequence: zero them once the tile lands, then
+                            // release the tile to the MMA thread through this stage's tail barrier
+                            if (!mbar_wait(full_bar(st), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
+                            uint8_t* vt = sgen + (sKV - sb) + st * TILE;
+                            const int r0 = it.Lkv - j * 128;  // rows of the partially valid box past Lkv
+                            const int r1 = min(128, (r0 + p.box_rows - 1) / p.box_rows * p.box_rows);
+                            for (int r = r0; r < r1; ++r)
+                                for (int c = 0; c < (D / 64) * 8; ++c)
+                                    *reinterpret_cast<uint4*>(vt + (r >> 3) * (D / 64) * 1024 + (c >> 3) * 1024 +
+                                                              (r & 7) * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
+                            fence_proxy_async_smem();
+                            mbar_arrive(b_vtail0 + 8 * st);
+                        }
+                    } else {
+                        tma_load_5d(sKV + st * TILE, map, full_bar(st), 0, it.kv_tok0 + j * 128, 0, g, it.batch);
+                    }
                     ++kv_it;
                 }
             }
@@ -261,8 +326,12 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
         int pr_cnt0 = 0, pr_cnt1 = 0, oe_cnt0 = 0, oe_cnt1 = 0;
         bool ok = true;
         const SmemDesc dQ = smem_desc_sw128_split(sQ, 16, 1024);
-        const SmemDesc dK = smem_desc_sw128_split(sKV, 16, 1024);
-        const SmemDesc dV = smem_desc_sw128_split(sKV, 16384, 1024);
+        // K/V tiles: [64-column block][128 rows] (8-row groups 1 KB apart), or in mode 2
+        // [8-row group][block][8 rows] (groups (D/64) KB apart, blocks 1 KB apart)
+        constexpr uint32_t NBK = D / 64;
+        const SmemDesc dK = smem_desc_sw128_split(sKV, 16, PAGED ? NBK * 1024 : 1024);
+        const SmemDesc dV = smem_desc_sw128_split(sKV, PAGED ? 1024 : 16384, PAGED ? NBK * 1024 : 1024);
+        uint32_t tail_par = 0;  // mode 2: per-stage parity of the tail barriers
         auto issue_qk = [&](int s, int st) {
             const uint32_t d_tmem = tmem + 128u * s;
             const SmemDesc a0{dQ.lo + ((s * TILE) >> 4), dQ.hi};
@@ -270,7 +339,8 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
-                tc_mma_ss(d_tmem, desc_at(a0, off), desc_at(b0, off), IDESC_QK, kk > 0 ? 1u : 0u);
+                const uint32_t offk = PAGED ? (kk >> 2) * 1024u + (kk & 3) * 32u : off;
+                tc_mma_ss(d_tmem, desc_at(a0, off), desc_at(b0, offk), IDESC_QK, kk > 0 ? 1u : 0u);
             }
         };
         auto issue_pv = [&](int s, int st, bool acc) {
@@ -279,7 +349,8 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
             const SmemDesc b0{dV.lo + ((st * TILE) >> 4), dV.hi};
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                tc_mma_ts(d_tmem, a_tmem + kk * 8u, desc_at(b0, kk * 2048u), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+                const uint32_t offv = PAGED ? kk * (2u * NBK * 1024u) : kk * 2048u;
+                tc_mma_ts(d_tmem, a_tmem + kk * 8u, desc_at(b0, offv), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
             }
         };
         for (int k = 0; ok; ++k) {
@@ -304,6 +375,10 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
             for (int j = 0; ok && j < it.n_kv; ++j) {
                 const int stV = kv_it % NST;
                 if (!mbar_wait(full_bar(stV), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
+                if (PAGED && paged_tile_has_tail(p, j * 128, it.Lkv)) {
+                    if (!mbar_wait(b_vtail0 + 8 * stV, (tail_par >> stV) & 1u, abort_flag)) { ok = false; break; }
+                    tail_par ^= 1u << stV;
+                }
                 ++kv_it;
                 const bool more = (j + 1 < it.n_kv);
                 const int stK1 = kv_it % NST;

@@ -137,3 +137,28 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(rsd, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         rsd.lib()
+
+
+def test_paged_prefill_rejects_bad_args_on_host(lib):
+    f = lib.attn_fwd_paged_prefill
+    fake = ctypes.c_void_p(0x100000)
+    q2 = L2(32 * 128, 128)
+    kp = L3(4 * 64 * 128, 128, 64 * 128)          # HND [pages, 4 heads, 64 rows, 128]
+    args = dict(B=2, Hq=32, Hkv=4, D=128, ps=64, P=100, maxkv=4096, maxsq=512, Tq=600, ks=kp, ws=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(fake, fake, fake, fake, None, fake, fake, 64, fake, a["B"], a["maxsq"], a["Tq"], a["Hq"],
+                 a["Hkv"], a["D"], a["ps"], a["P"], a["maxkv"], q2, q2, a["ks"], a["ks"],
+                 rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, a["ws"], 1 << 30 if a["ws"] else 0, None)
+
+    assert call() == rsd.ATTN_ERR_WORKSPACE                 # the work list needs a workspace
+    assert call(D=96) == rsd.ATTN_ERR_UNSUPPORTED
+    assert call(ps=48) == rsd.ATTN_ERR_UNSUPPORTED          # neither divides nor is divided by 128
+    assert call(ps=4) == rsd.ATTN_ERR_UNSUPPORTED           # fewer rows than one 8-row group
+    assert call(Hkv=5) == rsd.ATTN_ERR_INVALID_ARG          # 32 % 5 != 0
+    # a page stride that is not a whole number of 8-row groups
+    assert call(ks=L3(4 * 64 * 128 + 8, 128, 64 * 128)) == rsd.ATTN_ERR_UNSUPPORTED
+    assert call(B=0) == rsd.ATTN_OK                          # nothing to do
+    assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 32, 4) == \
+        rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 32, 4)

@@ -1,0 +1,115 @@
+"""Ragged queries over a paged K/V cache (chunked prefill, multi-token decode)
+on the GPU vs the fp64 oracle.  The oracle sees the same keys gathered out of
+the pool into contiguous per-sequence K/V by this test (numpy indexing), and
+the ragged oracle's bottom-right causal rule.  Also: bit-identical to the
+ragged kernel over that gathered K/V, NaN in the unused slots of a last page,
+empty caches and queries without keys."""
+import numpy as np
+import pytest
+import torch
+
+import ragged_scaled_dot_b200 as rsd
+import synth
+from gpu_util import assert_lse_close, assert_o_close, bits, gather_ragged, orc, ragged_gpu, ragged_rows_all
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _inputs(lens_q, lens_kv, Hq, Hkv, D, ps, seed, layout="HND"):
+    table, total = synth.page_table(lens_kv, ps, seed)
+    P = total + 2
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    q = synth.normal_bf16((int(cu_q[-1]), Hq, D), seed + 1, "cpu").to(DEV)
+    shape = (P, Hkv, ps, D) if layout == "HND" else (P, ps, Hkv, D)
+    k = synth.normal_bf16(shape, seed + 2, "cpu").to(DEV)
+    v = synth.normal_bf16(shape, seed + 3, "cpu").to(DEV)
+    return q, k, v, table, np.asarray(lens_kv, dtype=np.int32), cu_q
+
+
+def _gather(pool, table, lens_kv, ps, layout):
+    """Contiguous THD [sum kv, Hkv, D] copy of each sequence's keys, by page table."""
+    parts = []
+    for b, L in enumerate(lens_kv):
+        j = np.arange(int(L))
+        pages = torch.as_tensor(table[b, j // ps].astype(np.int64), device=pool.device)
+        slots = torch.as_tensor(j % ps, device=pool.device)
+        parts.append(pool[pages, :, slots] if layout == "HND" else pool[pages, slots])
+    Hkv, D = (pool.shape[1], pool.shape[3]) if layout == "HND" else (pool.shape[2], pool.shape[3])
+    if not parts:
+        return torch.zeros((0, Hkv, D), dtype=pool.dtype, device=pool.device)
+    return torch.cat(parts, 0).contiguous()
+
+
+def _run(q, k, v, table, kl, cu_q, ps, scale, causal, layout="HND", lse_layout=rsd.ATTN_LSE_PADDED_BSH):
+    B = len(cu_q) - 1
+    max_sq = max(1, int(np.max(np.diff(cu_q))))
+    Hq = q.shape[1]
+    o = torch.full((q.shape[0], Hq, v.shape[-1]), float("nan"), dtype=torch.bfloat16, device=DEV)
+    if lse_layout == rsd.ATTN_LSE_PADDED_BSH:
+        lse = torch.full((B, max_sq, Hq), float("nan"), dtype=torch.float32, device=DEV)
+    else:
+        lse = torch.full((q.shape[0], Hq), float("nan"), dtype=torch.float32, device=DEV)
+    Hkv = k.shape[1] if layout == "HND" else k.shape[2]
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(B, max_sq, q.shape[0], Hq, Hkv),
+                     dtype=torch.uint8, device=DEV)
+    rsd.attn_fwd_paged_prefill(
+        q, k, v, o, lse, torch.as_tensor(cu_q, device=DEV), torch.as_tensor(table, device=DEV),
+        torch.as_tensor(kl, device=DEV), max_seqlen_q=max_sq, page_size=ps,
+        max_kv_len=max(1, int(np.max(kl))), scale=scale, causal=causal, workspace=ws,
+        lse_layout=lse_layout, kv_layout=layout)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    return o, lse
+
+
+CASES = [
+    # (lens_q, lens_kv, Hq, Hkv, D, ps, layout, causal)
+    ([1, 2, 4, 100, 129], [1000, 64, 300, 100, 2000], 16, 4, 128, 64, "HND", True),   # MTP + chunks
+    ([37, 256, 5], [300, 700, 77], 8, 1, 64, 16, "NHD", False),
+    ([512, 300], [4096, 1024], 8, 2, 128, 128, "HND", True),                          # chunked prefill
+    ([9, 130], [40, 333], 4, 4, 128, 8, "NHD", True),                                   # 8-row pages
+    ([64, 200], [1500, 999], 16, 2, 64, 256, "HND", True),                              # 128-row boxes
+    ([100, 3], [40, 0], 4, 1, 128, 32, "HND", True),                                    # Lq > Lkv, empty cache
+]
+
+
+@pytest.mark.parametrize("lens_q,lens_kv,Hq,Hkv,D,ps,layout,causal", CASES)
+def test_paged_prefill_vs_oracle(lens_q, lens_kv, Hq, Hkv, D, ps, layout, causal):
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, Hq, Hkv, D, ps, seed=ps + Hq + len(lens_q), layout=layout)
+    scale = 1.0 / np.sqrt(D)
+    o, lse = _run(q, k, v, table, kl, cu_q, ps, scale, causal, layout)
+    kc, vc = _gather(k, table, kl, ps, layout), _gather(v, table, kl, ps, layout)
+    cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
+    rows = ragged_rows_all(cu_q, Hq)
+    o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(kc), bits(vc), cu_q, cu_kv, Hq, Hkv, scale, causal, rows)
+    og, lg = gather_ragged(o, lse, cu_q, rows, rsd.ATTN_LSE_PADDED_BSH)
+    where = f"paged prefill {lens_q}/{lens_kv} ps{ps} {layout} causal={causal}"
+    assert_o_close(og, o_ref, where)
+    assert_lse_close(lg, l_ref, where)
+
+
+def test_paged_prefill_matches_ragged_over_gathered_kv_bitwise():
+    lens_q, lens_kv, ps = [128, 300, 1], [1024, 300, 777], 64
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 16, 4, 128, ps, seed=5)
+    o1, l1 = _run(q, k, v, table, kl, cu_q, ps, 0.09, True, lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    kc, vc = _gather(k, table, kl, ps, "HND"), _gather(v, table, kl, ps, "HND")
+    cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
+    o2, l2 = ragged_gpu(q, kc, vc, cu_q, cu_kv, int(max(lens_q)), int(max(lens_kv)), 0.09, True,
+                        lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("ps", [16, 64])
+def test_paged_prefill_nan_past_kv_len_is_never_used(ps):
+    lens_q, lens_kv = [50, 7], [170, 90]
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=11)
+    kn, vn = k.clone(), v.clone()
+    for b, L in enumerate(lens_kv):
+        last = table[b, (L - 1) // ps]
+        kn[last, :, L % ps:] = float("nan")
+        vn[last, :, L % ps:] = float("nan")
+    o1, l1 = _run(q, k, v, table, kl, cu_q, ps, 0.1, True)
+    o2, l2 = _run(q, kn, vn, table, kl, cu_q, ps, 0.1, True)
+    assert torch.isfinite(o2.float()).all()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
