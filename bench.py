@@ -211,6 +211,30 @@ def make_dense_prefill(torch, rsd, synth, dev, seed_offset, B=0):
     return Part("dense_prefill", "TFLOP/s", flops / 1e12, 1, step, None, info), None
 
 
+def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
+    w = _with_batch(synth, synth.WORKLOADS["paged_prefill"], B)
+    L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
+    q, kp, vp, table, kl, cu_q, lq = synth.make_paged_prefill(w, dev, kv_lens=L)
+    T = q.shape[0]
+    smax = int(lq.max())
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, smax, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv), dtype=torch.uint8,
+                     device=dev)
+    cud = torch.as_tensor(cu_q, device=dev)
+    pt = torch.as_tensor(table, device=dev)
+    kld = torch.as_tensor(kl, device=dev)
+    maxL = int(L.max())
+
+    def step():
+        rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, cud, pt, kld, max_seqlen_q=smax, page_size=w.page_size,
+                                   max_kv_len=maxL, scale=w.scale, causal=True, workspace=ws)
+    flops = prefill_flops(lq, L, w.Hq, w.Dqk)
+    info = {"workload": w.notes, "flop_per_step": flops, "query_tokens": int(T),
+            "kv_tokens": int(L.sum()), "total_pages": int(kp.shape[0])}
+    return Part("paged_prefill", "TFLOP/s", flops / 1e12, 3, step, None, info), None
+
+
 def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
     w = _with_batch(synth, synth.WORKLOADS[name], B)
     L = synth.uniform_lengths(w.B, *w.len_range, w.seed + seed_offset)
@@ -421,6 +445,7 @@ def run_ours(args):
     extras = []
     if not args.no_extras:
         extras.append(make_dense_prefill(torch, rsd, synth, dev, off)[0])
+        extras.append(make_paged_prefill(torch, rsd, synth, dev, off)[0])
         mla, _ = make_paged(torch, rsd, synth, dev, off, "mla_decode", num_sms)
         extras.append(mla)
     torch.cuda.synchronize()
@@ -546,6 +571,8 @@ def run_one(args):
         part = make_ragged_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
     elif args.only == "dense_prefill":
         part = make_dense_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
+    elif args.only == "paged_prefill":
+        part = make_paged_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
     else:
         part = make_paged(torch, rsd, synth, "cuda", 0, args.only, num_sms, args.batch)[0]
     total_ms, per = time_part(torch, part, args.steps, args.warmup, None, 1)
@@ -604,7 +631,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "mla_decode"],
+    ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "paged_prefill",
+                                       "mla_decode"],
                     help="profiling: time one part only and print its own line")
     ap.add_argument("--batch", type=int, default=0, help="profiling: override the part's batch size")
     args = ap.parse_args()

@@ -114,6 +114,11 @@ WORKLOADS = {
         "paged_decode", "paged", seed=4, B=128, Hq=64, Hkv=8, Dqk=128, Dv=128,
         len_range=(1024, 32768), page_size=64, causal=False,
         notes="paged decode B=128 kv U[1024, 32768] page 64, H=64/8 D=128"),
+    "paged_prefill": Workload(
+        "paged_prefill", "paged", seed=6, B=16, Hq=32, Hkv=8, Dqk=128, Dv=128,
+        lengths=(1024,), len_range=(8192, 65536), page_size=64, causal=True,
+        notes="chunked prefill: 16 sequences, a 1024-token chunk at the end of a paged cache of "
+              "U[8192, 65536] keys, page 64, H=32/8 D=128, bottom-right causal"),
     "mla_decode": Workload(
         "mla_decode", "paged", seed=5, B=64, Hq=128, Hkv=1, Dqk=576, Dv=512,
         len_range=(4096, 65536), page_size=64, causal=False, v_aliases_k=True,
@@ -141,6 +146,21 @@ def make_dense(w: Workload, device="cpu", S=None, B=None):
     k = normal_bf16((B, S, w.Hkv, w.Dqk), w.seed * 10 + 2, device)
     v = normal_bf16((B, S, w.Hkv, w.Dv), w.seed * 10 + 3, device)
     return q, k, v
+
+
+def make_paged_prefill(w: Workload, device="cpu", kv_lens=None):
+    """Chunked-prefill inputs: q [B * chunk, Hq, D] packed (chunk = w.lengths[0]
+    queries per sequence), HND pools, page table (host), kv_lens (host), cu_q."""
+    L = np.asarray(kv_lens if kv_lens is not None else
+                   uniform_lengths(w.B, w.len_range[0], w.len_range[1], w.seed), dtype=np.int64)
+    chunk = int(w.lengths[0])
+    lq = np.minimum(L, chunk)
+    cu_q = cu_seqlens(lq)
+    table, total = page_table(L, w.page_size, w.seed)
+    q = normal_bf16((int(cu_q[-1]), w.Hq, w.Dqk), w.seed * 10 + 1, device)
+    k_pool = normal_bf16((total, w.Hkv, w.page_size, w.Dqk), w.seed * 10 + 2, device)
+    v_pool = normal_bf16((total, w.Hkv, w.page_size, w.Dv), w.seed * 10 + 3, device)
+    return q, k_pool, v_pool, table, L.astype(np.int32), cu_q, lq
 
 
 def make_paged(w: Workload, device="cpu", kv_lens=None, extra_pages: int = 0):

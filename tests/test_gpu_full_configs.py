@@ -100,3 +100,39 @@ def test_paged_decode_full_size(name):
     r = torch.as_tensor(rows.astype(np.int64), device=DEV)
     assert_o_close(o[r[:, 0], r[:, 1]], o_ref, f"{name} full (splits {S})")
     assert_lse_close(lse[r[:, 0], r[:, 1]], l_ref, f"{name} full (splits {S})")
+
+
+def test_paged_prefill_full_size():
+    """Chunked prefill at full size: 16 x 1024 queries over paged caches of up to
+    64k keys, vs the oracle over each sampled sequence's keys gathered from the pool."""
+    w = synth.WORKLOADS["paged_prefill"]
+    q, kp, vp, table, kl, cu_q, lq = synth.make_paged_prefill(w, DEV)
+    T, smax = q.shape[0], int(lq.max())
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((w.B, smax, w.Hq), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv), dtype=torch.uint8,
+                     device=DEV)
+    rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, torch.as_tensor(cu_q, device=DEV),
+                               torch.as_tensor(table, device=DEV), torch.as_tensor(kl, device=DEV),
+                               max_seqlen_q=smax, page_size=w.page_size, max_kv_len=int(kl.max()),
+                               scale=w.scale, causal=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    assert not torch.isnan(o).any()
+    rng = np.random.default_rng(2)
+    for b in (0, 7, 15):
+        L, n = int(kl[b]), int(lq[b])
+        j = np.arange(L)
+        pages = torch.as_tensor(table[b, j // w.page_size].astype(np.int64), device=DEV)
+        slots = torch.as_tensor(j % w.page_size, device=DEV)
+        kc, vc = kp[pages, :, slots].contiguous(), vp[pages, :, slots].contiguous()
+        rows = [(0, int(rng.integers(w.Hq)), i) for i in (0, 127, 128, n - 1)]
+        rows += [(0, int(rng.integers(w.Hq)), int(rng.integers(n))) for _ in range(60)]
+        rows = np.array(rows, dtype=np.int32)
+        q_b = q[int(cu_q[b]):int(cu_q[b + 1])]
+        o_ref, l_ref = orc().attn_ragged_rows(bits(q_b), bits(kc), bits(vc), np.array([0, n]),
+                                              np.array([0, L]), w.Hq, w.Hkv, w.scale, True, rows)
+        tok = torch.as_tensor(rows[:, 2].astype(np.int64) + int(cu_q[b]), device=DEV)
+        hh = torch.as_tensor(rows[:, 1].astype(np.int64), device=DEV)
+        assert_o_close(o[tok, hh], o_ref, f"paged prefill full b={b}")
+        assert_lse_close(lse[b, tok - int(cu_q[b]), hh], l_ref, f"paged prefill full b={b}")
