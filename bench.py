@@ -41,8 +41,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (profiles/), as a ratio to the bytes that scale with the launch, applied to
 # the full launch.  None when the kernel changed after the counters were taken.
 #   paged_decode: per K/V byte, profiles/decode_gqa_kernel_paged_b32.md (2.692 / 2.673 GB)
-#   ragged_prefill: per Q+K+V+O byte, profiles/prefill_kernel_ragged_b16.md (1.042 / 1.061 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.982, "paged_decode": 1.0071}
+#   ragged_prefill: per Q+K+V+O byte, profiles/prefill_kernel_ragged_b16.md (1.045 / 1.061 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.984, "paged_decode": 1.0071}
 
 
 def load_peaks():
