@@ -453,19 +453,11 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     tc_fence_after();
                     float x[128];
                     {
-                        uint32_t u0[32], u1[32], u2[32], u3[32];
-                        tmem_ld32(tS, u0);
-                        tmem_ld32(tS + 32u, u1);
-                        tmem_ld32(tS + 64u, u2);
-                        tmem_ld32(tS + 96u, u3);
+                        uint32_t u[128];
+                        tmem_ld128(tS, u);
                         tc_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            x[e] = __uint_as_float(u0[e]);
-                            x[32 + e] = __uint_as_float(u1[e]);
-                            x[64 + e] = __uint_as_float(u2[e]);
-                            x[96 + e] = __uint_as_float(u3[e]);
-                        }
+                        for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
                     }
                     const int kb = j * 128;
                     const bool masked = (kb + 128 > lim);
@@ -506,9 +498,10 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     const float2 sc2 = make_float2(sl2, sl2);
                     const float2 nm2 = make_float2(-mref, -mref);
                     float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
+                    uint32_t pk64[64];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        uint32_t pk[16];
+                        uint32_t* pk = pk64 + 16 * c;
 #pragma unroll
                         for (int e = 0; e < 16; ++e) {
                             const int col = 32 * c + 2 * e;
@@ -528,8 +521,8 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                             else sum0 = fadd2(sum0, pv);
                             pk[e] = pack_bf16(pv.x, pv.y);
                         }
-                        tmem_st16(tS + 16u * c, pk);
                     }
+                    tmem_st64(tS, pk64);
                     l = l * alpha + ((sum0.x + sum0.y) + (sum1.x + sum1.y));
                     const bool need_o = (j > 0) && old_finite && (alpha != 1.f);
                     if (__any_sync(0xffffffffu, need_o)) {
