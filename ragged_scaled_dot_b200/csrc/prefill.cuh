@@ -105,14 +105,15 @@ __device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal)
 
 __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx, PrefillItem& it) {
     if (p.mode == 0) {
-        // dense: (batch, kv head, query tile longest first, head pair)
-        const int per_b = p.Hkv * p.n_qtiles * p.pairs_per_group;
-        it.b = idx / per_b;
-        int rem = idx - it.b * per_b;
-        const int g = rem / (p.n_qtiles * p.pairs_per_group);
-        rem -= g * p.n_qtiles * p.pairs_per_group;
-        const int t = rem / p.pairs_per_group;
-        const int pr = rem - t * p.pairs_per_group;
+        // dense: (query tile longest first, batch, kv head, head pair): the static
+        // round-robin assignment then hands out the longest items first
+        const int per_t = p.B * p.Hkv * p.pairs_per_group;
+        const int t = idx / per_t;
+        int rem = idx - t * per_t;
+        it.b = rem / (p.Hkv * p.pairs_per_group);
+        rem -= it.b * p.Hkv * p.pairs_per_group;
+        const int g = rem / p.pairs_per_group;
+        const int pr = rem - g * p.pairs_per_group;
         it.qt = p.causal ? (p.n_qtiles - 1 - t) : t;
         it.h0 = g * p.G + pr * p.heads_per_item;
         it.q_tok0 = it.qt * 128;
