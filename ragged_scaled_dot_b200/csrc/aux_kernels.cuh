@@ -12,7 +12,9 @@ namespace b2 {
 // THD, with zero host reads"; "cuDNN Frontend v1.32.0 Release Notes", native
 // THD metadata setup fused on the device, work prefixes).  One block:
 //   1. validate each sequence against the host-declared capacities;
-//   2. order sequences longest first (counting sort on query-tile count);
+//   2. order sequences most work first (counting sort on the number of
+//      (query tile, kv tile) steps, which with a paged cache of unequal
+//      lengths differs between sequences of equal query length);
 //   3. give each sequence a contiguous run of items, ordered
 //      (kv head, query tile longest first, head pair), so that the CTAs that
 //      take consecutive items read the same sequence-head's K/V from L2.
@@ -37,6 +39,14 @@ __device__ __forceinline__ bool ragged_seq_ok(const int32_t* cu_q, const int32_t
     return q0 >= 0 && kv_ok && lq >= 0 && lk >= 0 && lq <= max_sq && lk <= max_skv && (int64_t)q1 <= total_q;
 }
 
+// Sort key: (query tile, kv tile) steps of all query tiles of a sequence, capped.
+__device__ __forceinline__ int seq_cost_key(int lq, int lk, int causal) {
+    const int nqt = (lq + 127) >> 7;
+    int cost = 0;
+    for (int qt = 0; qt < nqt && cost < kSortBuckets - 1; ++qt) cost += prefill_n_kv(qt, lq, lk, causal);
+    return min(cost, kSortBuckets - 1);
+}
+
 __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv,
     const int32_t* __restrict__ kv_lens, int B, int max_sq,
@@ -53,14 +63,17 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         if (cu_q[0] != 0 || (kv_lens == nullptr && cu_kv[0] != 0)) record_status(ATTN_ERR_DEVICE_INPUT);
     }
     __syncthreads();
-    // 1. validate, histogram of query-tile counts
+    // 1. validate, histogram of the sort keys
     for (int b = tid; b < B; b += blockDim.x) {
-        int nqt = 0;
-        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv))
-            nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
-        else
+        int nqt = 0, key = 0;
+        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) {
+            const int lq = cu_q[b + 1] - cu_q[b];
+            nqt = (lq + 127) >> 7;
+            key = seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal);
+        } else {
             record_status(ATTN_ERR_DEVICE_INPUT);
-        atomicAdd(&hist[min(nqt, kSortBuckets - 1)], 1);
+        }
+        atomicAdd(&hist[key], 1);
         atomicAdd(&n_tiles_sh, nqt);
     }
     __syncthreads();
@@ -75,10 +88,13 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     }
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) {
-        int nqt = 0;
-        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv))
-            nqt = (cu_q[b + 1] - cu_q[b] + 127) >> 7;
-        const int r = atomicAdd(&hist[min(nqt, kSortBuckets - 1)], 1);
+        int nqt = 0, key = 0;
+        if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) {
+            const int lq = cu_q[b + 1] - cu_q[b];
+            nqt = (lq + 127) >> 7;
+            key = seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal);
+        }
+        const int r = atomicAdd(&hist[key], 1);
         rank_of[b] = r;
         sorted_nqt[r] = nqt;
     }
