@@ -330,14 +330,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | ((uint32_t)(M >> 4) << 24);
 }
 
-// Per-warpgroup register reallocation.  All four warps of a warpgroup must
-// execute the same instruction, and the block's total (threads x registers)
-// must not exceed what it was launched with.
-template <int N>
-__device__ __forceinline__ void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
-template <int N>
-__device__ __forceinline__ void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
-
 // ---------------------------------------------------------------------------
 // Math helpers
 // ---------------------------------------------------------------------------
