@@ -27,9 +27,8 @@
 // row.  Measured on B200, one SM streams about 220 GB/s with such boxes but
 // only 60 GB/s with boxes of one 64-column block (128-byte pieces of 1152-byte
 // rows) and 80 GB/s with three; the smaller boxes left the kernel load-bound.
-// Both CTAs
-// stream the same pages (the second read hits L2); page ids are fetched a
-// chunk ahead of the loads that use them.  Keys past the split's range read
+// Both CTAs stream the same pages (the second read hits L2); page ids are
+// fetched a chunk ahead of the loads that use them.  Keys past the split's range read
 // zeros (an out-of-range page coordinate); the value rows of the one
 // partially valid box are zeroed in shared memory, so 0 * NaN from stale
 // cache slots can not reach O.
