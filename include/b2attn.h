@@ -80,6 +80,15 @@ extern "C" {
                                    Notes", "New: the FlashInfer serving path runs
                                    on FROST": per-batch padded Stats seeded -inf) */
 #define ATTN_LSE_PACKED_TH   1  /* token-major [total_q, Hq]                    */
+#define ATTN_LSE_PACKED_HT   2  /* head-major [Hq, total_q] (row stride total_q),
+                                   FlashAttention's and PyTorch varlen's
+                                   softmax_lse ("cuDNN Frontend v1.30.0 Release
+                                   Notes", head-major [h, total_q] Stats)       */
+/* Flag OR-ed into lse_layout: write the LSE in base 2,
+ * log2(sum_j exp(s_j)) = LSE * log2(e), the convention of flash-attention-style
+ * consumers, instead of the natural log ("cuDNN Frontend v1.30.0 Release
+ * Notes", "New: stats_use_log2 -- LSE in base 2").  -inf stays -inf. */
+#define ATTN_LSE_LOG2        0x100
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *attn_status_string(int status);
@@ -115,7 +124,8 @@ int attn_fwd_dense(const void *q, const void *k, const void *v, void *o, float *
  * read or written ("cuDNN Frontend v1.28.0 release notes", "Updates to Graph
  * API / SDPA": max_total_seq_len_q / _kv).  A device table that breaks them
  * sets ATTN_ERR_DEVICE_INPUT and the offending sequences are skipped.
- * lse (nullable): layout per lse_layout (ATTN_LSE_PADDED_BSH or _PACKED_TH).
+ * lse (nullable): layout per lse_layout (ATTN_LSE_PADDED_BSH, _PACKED_TH or
+ * _PACKED_HT, optionally | ATTN_LSE_LOG2).
  * workspace: device scratch of at least attn_fwd_ragged_workspace_size(...)
  * bytes, 256-byte aligned; it holds the device-built work list.
  */
@@ -203,6 +213,28 @@ int attn_fwd_paged(const void *q, const void *k_pool, const void *v_pool, void *
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * attn_fwd_paged with independent K and V page tables: logical key t of
+ * sequence b reads its key row from page k_page_table[b*k_page_table_stride +
+ * t / page_size] of k_pool and its value row from page
+ * v_page_table[b*v_page_table_stride + t / page_size] of v_pool ("cuDNN
+ * Frontend v1.32.0 Release Notes", "SDPA: wider native forward support":
+ * independent K/V tables and layouts).  Both are DEVICE int32 tables whose
+ * rows cover max_kv_len keys; page ids of both lie in [0, num_pages) (each
+ * pool holds at least num_pages pages).  Everything else, including the MLA
+ * and GQA rules and the split-KV workspace, is as for attn_fwd_paged, which
+ * is this call with both tables the same.
+ */
+int attn_fwd_paged_kv_tables(const void *q, const void *k_pool, const void *v_pool, void *o,
+                             float *lse, const int32_t *k_page_table, int64_t k_page_table_stride,
+                             const int32_t *v_page_table, int64_t v_page_table_stride,
+                             const int32_t *kv_lens, int B, int Hq, int Hkv, int Dqk, int Dv,
+                             int page_size, int64_t num_pages, int max_kv_len,
+                             const int64_t q_strides[2], const int64_t o_strides[2],
+                             const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
+                             float scale, int num_splits,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Ragged queries over a paged K/V cache: chunked prefill and multi-token
  * decode ("cuDNN Frontend v1.31.0 Release Notes", "SDPA: paged KV, split-KV,
  * and engine selection": paged K/V for prefill; "cuDNN Frontend v1.28.0
@@ -231,6 +263,23 @@ int attn_fwd_paged_prefill(const void *q, const void *k_pool, const void *v_pool
                            const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
                            int lse_layout, float scale, int causal,
                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * attn_fwd_paged_prefill with independent K and V page tables (K rows through
+ * k_page_table, V rows through v_page_table, as for attn_fwd_paged_kv_tables);
+ * otherwise identical, and attn_fwd_paged_prefill is this call with both
+ * tables the same.
+ */
+int attn_fwd_paged_prefill_kv_tables(const void *q, const void *k_pool, const void *v_pool, void *o,
+                                     float *lse, const int32_t *cu_seqlens_q,
+                                     const int32_t *k_page_table, int64_t k_page_table_stride,
+                                     const int32_t *v_page_table, int64_t v_page_table_stride,
+                                     const int32_t *kv_lens, int B, int max_seqlen_q, int64_t total_q,
+                                     int Hq, int Hkv, int D, int page_size, int64_t num_pages,
+                                     int max_kv_len, const int64_t q_strides[2],
+                                     const int64_t o_strides[2], const int64_t k_pool_strides[3],
+                                     const int64_t v_pool_strides[3], int lse_layout, float scale,
+                                     int causal, void *workspace, size_t workspace_bytes, void *stream);
 
 /* Workspace bytes attn_fwd_paged_prefill needs (the work list of attn_fwd_ragged). */
 size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv);

@@ -26,6 +26,8 @@ ATTN_ERR_DEVICE_INPUT = 6
 ATTN_ERR_CUDA = 7
 ATTN_LSE_PADDED_BSH = 0
 ATTN_LSE_PACKED_TH = 1
+ATTN_LSE_PACKED_HT = 2
+ATTN_LSE_LOG2 = 0x100
 
 # every symbol include/b2attn.h declares: name -> (restype, argtypes)
 _I, _L, _F, _P, _Z, _U64 = (ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p,
@@ -44,9 +46,13 @@ SIGNATURES = {
     "attn_fwd_ragged_noalloc_max_scratch": (_Z, []),
     "attn_fwd_paged": (_I, [_P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _I, _I, _I, _I, _L, _I,
                             _L2, _L2, _L3, _L3, _F, _I, _P, _Z, _P]),
+    "attn_fwd_paged_kv_tables": (_I, [_P, _P, _P, _P, _P, _P, _L, _P, _L, _P, _I, _I, _I, _I, _I, _I, _L, _I,
+                                      _L2, _L2, _L3, _L3, _F, _I, _P, _Z, _P]),
     "attn_fwd_paged_workspace_size": (_Z, [_I, _I, _I, _I]),
     "attn_fwd_paged_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _L, _I, _I, _I, _I, _L, _I,
                                     _L2, _L2, _L3, _L3, _I, _F, _I, _P, _Z, _P]),
+    "attn_fwd_paged_prefill_kv_tables": (_I, [_P, _P, _P, _P, _P, _P, _P, _L, _P, _L, _P, _I, _I, _L, _I, _I,
+                                              _I, _I, _L, _I, _L2, _L2, _L3, _L3, _I, _F, _I, _P, _Z, _P]),
     "attn_fwd_paged_prefill_workspace_size": (_Z, [_I, _I, _L, _I, _I]),
     "attn_paged_suggest_splits": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "attn_split_merge": (_I, [_P, _P, _I, _L, _I, _P, _L, _P, _P]),
@@ -218,6 +224,27 @@ def attn_fwd_paged(q, k_pool, v_pool, o, lse, page_table, kv_lens, *, page_size:
         ws_bytes, _stream(stream)), "attn_fwd_paged")
 
 
+def attn_fwd_paged_kv_tables(q, k_pool, v_pool, o, lse, k_page_table, v_page_table, kv_lens, *,
+                             page_size: int, max_kv_len: int, scale: float, num_splits: int,
+                             workspace=None, kv_layout: str = "HND", stream=None):
+    """attn_fwd_paged with independent K and V page tables (int32 CUDA
+    [B, max_pages] each): key rows through k_page_table, value rows through
+    v_page_table."""
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (o, "o")):
+        _bf16(t, n)
+    B, Hq, Dqk = q.shape
+    Dv = o.shape[-1]
+    Hkv = k_pool.shape[1] if kv_layout == "HND" else k_pool.shape[2]
+    num_pages = min(k_pool.shape[0], v_pool.shape[0])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().attn_fwd_paged_kv_tables(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(o), _ptr(lse), _ptr(k_page_table),
+        int(k_page_table.stride(0)), _ptr(v_page_table), int(v_page_table.stride(0)), _ptr(kv_lens),
+        B, Hq, Hkv, Dqk, Dv, int(page_size), int(num_pages), int(max_kv_len), _L2(q.stride(0), q.stride(1)),
+        _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout), pool_strides(v_pool, kv_layout),
+        float(scale), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream)), "attn_fwd_paged_kv_tables")
+
+
 def attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv) -> int:
     return int(lib().attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv))
 
@@ -246,6 +273,29 @@ def attn_fwd_paged_prefill(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, 
         _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout), pool_strides(v_pool, kv_layout),
         int(lse_layout), float(scale), int(causal), _ptr(workspace), ws_bytes, _stream(stream)),
         "attn_fwd_paged_prefill")
+
+
+def attn_fwd_paged_prefill_kv_tables(q, k_pool, v_pool, o, lse, cu_seqlens_q, k_page_table, v_page_table,
+                                     kv_lens, *, max_seqlen_q: int, page_size: int, max_kv_len: int,
+                                     scale: float, causal: bool, workspace,
+                                     lse_layout: int = ATTN_LSE_PADDED_BSH, kv_layout: str = "HND",
+                                     total_q=None, stream=None):
+    """attn_fwd_paged_prefill with independent K and V page tables."""
+    for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (o, "o")):
+        _bf16(t, n)
+    B = cu_seqlens_q.numel() - 1
+    Hq, D = q.shape[1], q.shape[2]
+    Hkv = k_pool.shape[1] if kv_layout == "HND" else k_pool.shape[2]
+    num_pages = min(k_pool.shape[0], v_pool.shape[0])
+    total_q = q.shape[0] if total_q is None else total_q
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().attn_fwd_paged_prefill_kv_tables(
+        _ptr(q), _ptr(k_pool), _ptr(v_pool), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(k_page_table),
+        int(k_page_table.stride(0)), _ptr(v_page_table), int(v_page_table.stride(0)), _ptr(kv_lens), B,
+        int(max_seqlen_q), int(total_q), Hq, Hkv, D, int(page_size), int(num_pages), int(max_kv_len),
+        _L2(q.stride(0), q.stride(1)), _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout),
+        pool_strides(v_pool, kv_layout), int(lse_layout), float(scale), int(causal), _ptr(workspace), ws_bytes,
+        _stream(stream)), "attn_fwd_paged_prefill_kv_tables")
 
 
 # --------------------------------------------------------------------- merge

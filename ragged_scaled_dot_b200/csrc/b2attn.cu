@@ -305,7 +305,9 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     if (B < 0 || max_seqlen_q < 0 || max_seqlen_kv < 0 || total_q < 0 || total_kv < 0) return ATTN_ERR_INVALID_ARG;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
-    if (lse_layout != ATTN_LSE_PADDED_BSH && lse_layout != ATTN_LSE_PACKED_TH) return ATTN_ERR_INVALID_ARG;
+    const int lse_base = lse_layout & ~ATTN_LSE_LOG2;
+    if (lse_base != ATTN_LSE_PADDED_BSH && lse_base != ATTN_LSE_PACKED_TH && lse_base != ATTN_LSE_PACKED_HT)
+        return ATTN_ERR_INVALID_ARG;
     if (!q_strides || !k_strides || !v_strides || !o_strides) return ATTN_ERR_INVALID_ARG;
     if (Dqk != Dv || (Dqk != 64 && Dqk != 128)) return ATTN_ERR_UNSUPPORTED;
     if (total_q >= ((int64_t)1 << 31) || total_kv >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
@@ -347,7 +349,7 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
         hpi, G, header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
         max_tiles);
     if (int e = launch_status()) return e;
-    if (lse != nullptr && lse_layout == ATTN_LSE_PADDED_BSH) {
+    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
         const int64_t n = (int64_t)B * max_seqlen_q * Hq;
         const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
         b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
@@ -369,8 +371,10 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     pp.o_ts = o_strides[0];
     pp.o_hs = o_strides[1];
     pp.lse = lse;
-    pp.lse_layout = (lse_layout == ATTN_LSE_PADDED_BSH) ? 1 : 2;
+    pp.lse_layout = (lse_base == ATTN_LSE_PADDED_BSH) ? 1 : (lse_base == ATTN_LSE_PACKED_TH) ? 2 : 3;
     pp.lse_smax = max_seqlen_q;
+    pp.lse_hs = total_q;
+    pp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
     pp.scale_log2 = scale * kLog2e;
     pp.causal = causal;
     const int64_t items_max = (int64_t)max_tiles * n_pairs;
@@ -408,21 +412,41 @@ int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool
                            const int64_t o_strides[2], const int64_t k_pool_strides[3],
                            const int64_t v_pool_strides[3], int lse_layout, float scale, int causal,
                            void* workspace, size_t workspace_bytes, void* stream) {
+    return attn_fwd_paged_prefill_kv_tables(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, page_table_stride,
+                                            page_table, page_table_stride, kv_lens, B, max_seqlen_q, total_q, Hq,
+                                            Hkv, D, page_size, num_pages, max_kv_len, q_strides, o_strides,
+                                            k_pool_strides, v_pool_strides, lse_layout, scale, causal, workspace,
+                                            workspace_bytes, stream);
+}
+
+int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
+                                     const int32_t* cu_seqlens_q, const int32_t* k_page_table,
+                                     int64_t k_page_table_stride, const int32_t* v_page_table,
+                                     int64_t v_page_table_stride, const int32_t* kv_lens, int B, int max_seqlen_q,
+                                     int64_t total_q, int Hq, int Hkv, int D, int page_size, int64_t num_pages,
+                                     int max_kv_len, const int64_t q_strides[2], const int64_t o_strides[2],
+                                     const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
+                                     int lse_layout, float scale, int causal, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
     if (B < 0 || max_seqlen_q < 0 || total_q < 0 || max_kv_len < 0 || num_pages < 0) return ATTN_ERR_INVALID_ARG;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
-    if (lse_layout != ATTN_LSE_PADDED_BSH && lse_layout != ATTN_LSE_PACKED_TH) return ATTN_ERR_INVALID_ARG;
+    const int lse_base = lse_layout & ~ATTN_LSE_LOG2;
+    if (lse_base != ATTN_LSE_PADDED_BSH && lse_base != ATTN_LSE_PACKED_TH && lse_base != ATTN_LSE_PACKED_HT)
+        return ATTN_ERR_INVALID_ARG;
     if (!q_strides || !o_strides || !k_pool_strides || !v_pool_strides) return ATTN_ERR_INVALID_ARG;
-    if (page_size <= 0 || page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
+    if (page_size <= 0 || k_page_table_stride < 0 || v_page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     // a page box of min(page_size, 128) rows: whole 8-row groups that tile a 128-key tile
     if (!(page_size % 128 == 0 || (128 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
     if (total_q >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
     if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
-    if (!q || !k_pool || !v_pool || !o || !cu_seqlens_q || !page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
+    if (!q || !k_pool || !v_pool || !o || !cu_seqlens_q || !k_page_table || !v_page_table || !kv_lens)
+        return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     if (num_pages == 0) return ATTN_ERR_INVALID_ARG;
-    if (B > 1 && page_table_stride < ((int64_t)max_kv_len + page_size - 1) / page_size) return ATTN_ERR_INVALID_ARG;
+    const int64_t row_pages = ((int64_t)max_kv_len + page_size - 1) / page_size;
+    if (B > 1 && (k_page_table_stride < row_pages || v_page_table_stride < row_pages)) return ATTN_ERR_INVALID_ARG;
     for (int i = 0; i < 2; ++i)
         if (!stride_ok(q_strides[i]) || !stride_ok(o_strides[i])) return ATTN_ERR_INVALID_ARG;
     for (int i = 0; i < 3; ++i)
@@ -470,7 +494,7 @@ int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool
         header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
         max_tiles);
     if (int e = launch_status()) return e;
-    if (lse != nullptr && lse_layout == ATTN_LSE_PADDED_BSH) {
+    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
         const int64_t n = (int64_t)B * max_seqlen_q * Hq;
         const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
         b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
@@ -490,13 +514,17 @@ int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool
     pp.o_ts = o_strides[0];
     pp.o_hs = o_strides[1];
     pp.lse = lse;
-    pp.lse_layout = (lse_layout == ATTN_LSE_PADDED_BSH) ? 1 : 2;
+    pp.lse_layout = (lse_base == ATTN_LSE_PADDED_BSH) ? 1 : (lse_base == ATTN_LSE_PACKED_TH) ? 2 : 3;
     pp.lse_smax = max_seqlen_q;
+    pp.lse_hs = total_q;
+    pp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
     pp.scale_log2 = scale * kLog2e;
     pp.causal = causal;
     pp.kv_lens = kv_lens;
-    pp.page_table = page_table;
-    pp.pt_stride = page_table_stride;
+    pp.page_table = k_page_table;
+    pp.pt_stride = k_page_table_stride;
+    pp.v_page_table = v_page_table;
+    pp.v_pt_stride = v_page_table_stride;
     pp.page_size = page_size;
     pp.box_rows = R;
     pp.num_pages = num_pages;
@@ -552,10 +580,23 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
                    const int64_t q_strides[2], const int64_t o_strides[2], const int64_t k_pool_strides[3],
                    const int64_t v_pool_strides[3], float scale, int num_splits, void* workspace,
                    size_t workspace_bytes, void* stream) {
+    return attn_fwd_paged_kv_tables(q, k_pool, v_pool, o, lse, page_table, page_table_stride, page_table,
+                                    page_table_stride, kv_lens, B, Hq, Hkv, Dqk, Dv, page_size, num_pages,
+                                    max_kv_len, q_strides, o_strides, k_pool_strides, v_pool_strides, scale,
+                                    num_splits, workspace, workspace_bytes, stream);
+}
+
+int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
+                             const int32_t* k_page_table, int64_t k_page_table_stride,
+                             const int32_t* v_page_table, int64_t v_page_table_stride, const int32_t* kv_lens,
+                             int B, int Hq, int Hkv, int Dqk, int Dv, int page_size, int64_t num_pages,
+                             int max_kv_len, const int64_t q_strides[2], const int64_t o_strides[2],
+                             const int64_t k_pool_strides[3], const int64_t v_pool_strides[3], float scale,
+                             int num_splits, void* workspace, size_t workspace_bytes, void* stream) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_kv_len < 0 || num_pages < 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || num_splits < 1 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
     if (!q_strides || !o_strides || !k_pool_strides || !v_pool_strides) return ATTN_ERR_INVALID_ARG;
-    if (page_size <= 0 || page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
+    if (page_size <= 0 || k_page_table_stride < 0 || v_page_table_stride < 0) return ATTN_ERR_INVALID_ARG;
     const int G = Hq / Hkv;
     const bool mla = (Dqk == 576 && Dv == 512);
     const bool gqa = (Dqk == Dv && (Dqk == 64 || Dqk == 128) && G <= 16);
@@ -567,11 +608,12 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     if (!(page_size % 64 == 0 || (64 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
     if (B > 65535 || Hkv > 65535 || num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
     if (B == 0) return ATTN_OK;
-    if (!q || !k_pool || !v_pool || !o || !page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
+    if (!q || !k_pool || !v_pool || !o || !k_page_table || !v_page_table || !kv_lens) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     if (num_pages == 0) return ATTN_ERR_INVALID_ARG;
-    // every row of the page table must cover max_kv_len keys
-    if (B > 1 && page_table_stride < ((int64_t)max_kv_len + page_size - 1) / page_size) return ATTN_ERR_INVALID_ARG;
+    // every row of each page table must cover max_kv_len keys
+    const int64_t row_pages = ((int64_t)max_kv_len + page_size - 1) / page_size;
+    if (B > 1 && (k_page_table_stride < row_pages || v_page_table_stride < row_pages)) return ATTN_ERR_INVALID_ARG;
     for (int i = 0; i < 2; ++i)
         if (!stride_ok(q_strides[i]) || !stride_ok(o_strides[i])) return ATTN_ERR_INVALID_ARG;
     for (int i = 0; i < 3; ++i)
@@ -611,8 +653,10 @@ int attn_fwd_paged(const void* q, const void* k_pool, const void* v_pool, void* 
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.q_bs = q_strides[0];
     dp.q_hs = q_strides[1];
-    dp.page_table = page_table;
-    dp.pt_stride = page_table_stride;
+    dp.page_table = k_page_table;
+    dp.pt_stride = k_page_table_stride;
+    dp.v_page_table = v_page_table;
+    dp.v_pt_stride = v_page_table_stride;
     dp.kv_lens = kv_lens;
     dp.B = B;
     dp.Hq = Hq;

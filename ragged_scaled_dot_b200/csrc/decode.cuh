@@ -25,8 +25,10 @@ struct DecodeParams {
     CUtensorMap tm_v;
     const __nv_bfloat16* q;
     int64_t q_bs, q_hs;
-    const int32_t* page_table;
+    const int32_t* page_table;  // K pages
     int64_t pt_stride;
+    const int32_t* v_page_table;  // V pages (the K table unless the caller gives its own)
+    int64_t v_pt_stride;
     const int32_t* kv_lens;
     int B, Hq, Hkv, G;
     int page_size, box_rows;  // rows per TMA box: min(page_size, chunk keys)
@@ -67,14 +69,16 @@ __device__ __forceinline__ uint32_t decode_chunk_bytes(const DecodeParams& p, in
 }
 
 // Issues the TMA loads of that chunk for kv head g of sequence b: rows
-// [r, r + box_rows) of the chunk come from one page (page-table lookup).
+// [r, r + box_rows) of the chunk come from one page (lookup in `table`, the K
+// or the V page table).
 __device__ __forceinline__ void decode_issue_chunk(const DecodeParams& p, const CUtensorMap* map,
+                                                   const int32_t* table, int64_t table_stride,
                                                    uint32_t dst, uint32_t bar, int b, int g, int t0,
                                                    int hi, int ncol_blocks, uint32_t block_bytes) {
     const int nkeys = min(64, hi - t0);
     for (int r = 0; r < nkeys; r += p.box_rows) {
         const int t = t0 + r;
-        int page = __ldg(p.page_table + (int64_t)b * p.pt_stride + t / p.page_size);
+        int page = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
         if (page < 0 || (int64_t)page >= p.num_pages) {
             record_status(ATTN_ERR_DEVICE_INPUT);
             page = -1;  // out of range: TMA fills the box with zeros
@@ -141,8 +145,10 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 const int t0 = lo + c * 64;
                 mbar_arrive_expect_tx(full_bar(st), decode_chunk_bytes(p, t0, hi, C::NCB, 2));
                 const uint32_t dst = sb + st * C::STAGE;
-                decode_issue_chunk(p, &p.tm_k, dst, full_bar(st), b, g, t0, hi, C::NCB, C::BLK);
-                decode_issue_chunk(p, &p.tm_v, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK);
+                decode_issue_chunk(p, &p.tm_k, p.page_table, p.pt_stride, dst, full_bar(st), b, g, t0, hi, C::NCB,
+                                   C::BLK);
+                decode_issue_chunk(p, &p.tm_v, p.v_page_table, p.v_pt_stride, dst + C::CHUNK, full_bar(st), b, g,
+                                   t0, hi, C::NCB, C::BLK);
             }
             // drain: every issued load lands before the block leaves
             for (int c = max(0, n_chunks - NST); c < n_chunks; ++c)

@@ -93,15 +93,15 @@ static_assert(9 % MlaTcCfg::KB == 0 && 8 % MlaTcCfg::VB == 0 && MlaTcCfg::VB % 2
 // loads are only issued here; the producer fetches the next chunk's ids while
 // it issues the current chunk's boxes.  Bit i of the result: box i holds keys
 // of the split.
-__device__ __forceinline__ uint32_t mla_fetch_pages(const DecodeParams& p, int b, int t0, int hi, int np,
-                                                    int (&pg)[4]) {
+__device__ __forceinline__ uint32_t mla_fetch_pages(const DecodeParams& p, const int32_t* table, int64_t table_stride,
+                                                    int b, int t0, int hi, int np, int (&pg)[4]) {
     uint32_t live = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int t = t0 + i * p.box_rows;
         pg[i] = -1;
         if (i < np && t < hi) {
-            pg[i] = __ldg(p.page_table + (int64_t)b * p.pt_stride + t / p.page_size);
+            pg[i] = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
             live |= 1u << i;
         }
     }
@@ -205,7 +205,8 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
         if (warp == 0 && lane == 0) {
             prefetch_tmap(&p.tm_k);
             int pc[4], pn[4];
-            uint32_t lc = 0, ln = (n_chunks > 0) ? mla_fetch_pages(p, b, lo, hi, np, pn) : 0u;
+            uint32_t lc = 0;
+            uint32_t ln = (n_chunks > 0) ? mla_fetch_pages(p, p.page_table, p.pt_stride, b, lo, hi, np, pn) : 0u;
             int ki = 0;
             bool ok = true;
             for (int j = 0; ok && j < n_chunks; ++j) {
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 4; ++i) pc[i] = pn[i];
                 lc = ln;
-                if (j + 1 < n_chunks) ln = mla_fetch_pages(p, b, t0 + 64, hi, np, pn);
+                if (j + 1 < n_chunks) ln = mla_fetch_pages(p, p.page_table, p.pt_stride, b, t0 + 64, hi, np, pn);
                 for (int t = 0; t < C::KLOADS; ++t) {
                     const int st = ki % C::RK;
                     if (!mbar_wait(sBar + C::B_KEMPTY + 8 * st, ((ki / C::RK) & 1) ^ 1, abort_flag)) {
@@ -431,7 +432,8 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
         if (warp == 0 && lane == 0) {
             prefetch_tmap(&p.tm_v);
             int pc[4], pn[4];
-            uint32_t lc = 0, ln = (n_chunks > 0) ? mla_fetch_pages(p, b, lo, hi, np, pn) : 0u;
+            uint32_t lc = 0;
+            uint32_t ln = (n_chunks > 0) ? mla_fetch_pages(p, p.v_page_table, p.v_pt_stride, b, lo, hi, np, pn) : 0u;
             int vi = 0;
             bool ok = true;
             for (int j = 0; ok && j < n_chunks; ++j) {
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 4; ++i) pc[i] = pn[i];
                 lc = ln;
-                if (j + 1 < n_chunks) ln = mla_fetch_pages(p, b, t0 + 64, hi, np, pn);
+                if (j + 1 < n_chunks) ln = mla_fetch_pages(p, p.v_page_table, p.v_pt_stride, b, t0 + 64, hi, np, pn);
                 for (int hf = 0; hf < C::VLOADS; ++hf) {
                     const int st = vi % C::RV;
                     const uint32_t full = sBar + C::B_VFULL + 8 * st;

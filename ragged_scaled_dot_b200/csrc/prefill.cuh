@@ -68,16 +68,20 @@ struct PrefillParams {
     __nv_bfloat16* o;
     int64_t o_bs, o_ts, o_hs;  // element strides (batch, token, head)
     float* lse;
-    int lse_layout;  // 0 dense [B,Hq,Sq], 1 padded [B,smax,Hq], 2 packed [T,Hq]
+    int lse_layout;  // 0 dense [B,Hq,Sq], 1 padded [B,smax,Hq], 2 packed [T,Hq], 3 packed [Hq,T]
     int lse_smax;
+    int64_t lse_hs;  // layout 3: row stride (declared total_q)
+    int lse_log2;    // 1: LSE in base 2
     float scale_log2;
     int causal;
     // mode 2 (queries of a ragged batch over a paged K/V cache): key t of
     // sequence b is row t % page_size of page page_table[b * pt_stride + t / page_size];
     // the pool maps address 8-row groups: group = page * groups_per_page + row / 8
     const int32_t* kv_lens;
-    const int32_t* page_table;
+    const int32_t* page_table;  // K pages
     int64_t pt_stride;
+    const int32_t* v_page_table;  // V pages (the K table unless the caller gives its own)
+    int64_t v_pt_stride;
     int page_size, box_rows;  // box_rows = min(page_size, 128) rows per page box
     int64_t num_pages;
     int groups_per_page;      // page stride / (8 x row stride) of the pool
@@ -149,13 +153,14 @@ __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx
 // [group][block][8 rows][128 B].  Two 64-row boxes placed back to back keep
 // one uniform 8-row-group stride, so the tile is a single MMA operand across
 // pages.  Boxes at or past Lkv (or with a bad page id, recorded) read zeros.
-__device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const CUtensorMap* map, uint32_t dst,
+__device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const CUtensorMap* map,
+                                                 const int32_t* table, int64_t table_stride, uint32_t dst,
                                                  uint32_t bar, int b, int g, int t0, int Lkv, uint32_t box_bytes) {
     for (int i = 0; i < 128 / p.box_rows; ++i) {
         const int t = t0 + i * p.box_rows;
         int gg = p.n_groups;
         if (t < Lkv) {
-            const int page = __ldg(p.page_table + (int64_t)b * p.pt_stride + t / p.page_size);
+            const int page = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
             if (page < 0 || (int64_t)page >= p.num_pages)
                 record_status(ATTN_ERR_DEVICE_INPUT);
             else
@@ -294,7 +299,8 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
                     if constexpr (PAGED) {
                         const uint32_t box_bytes = (uint32_t)p.box_rows * (D / 64) * 128u;
-                        paged_issue_tile(p, map, sKV + st * TILE, full_bar(st), it.b, g, j * 128, it.Lkv, box_bytes);
+                        paged_issue_tile(p, map, t ? p.v_page_table : p.page_table, t ? p.v_pt_stride : p.pt_stride,
+                                         sKV + st * TILE, full_bar(st), it.b, g, j * 128, it.Lkv, box_bytes);
                         if (t == 1 && paged_tile_has_tail(p, j * 128, it.Lkv)) {
                             // value rows past the sequence: zero them once the tile lands, then
                             // release the tile to the MMA thread through this stage's tail barrier
@@ -577,11 +583,14 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                 for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
             }
             if (valid && p.lse != nullptr) {
-                const float lse = (l > 0.f) ? (m_use + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                // m is kept in the log2 domain, so m + log2(l) is the base-2 LSE
+                const float lse2 = (l > 0.f) ? (m_use + log2f(l)) : -INFINITY;
+                const float lse = p.lse_log2 ? lse2 : lse2 * 0.6931471805599453f;
                 int64_t li;
                 if (p.lse_layout == 0) li = ((int64_t)it.b * p.Hq + h) * p.Sq + row;
                 else if (p.lse_layout == 1) li = ((int64_t)it.b * p.lse_smax + row) * p.Hq + h;
-                else li = (int64_t)tok * p.Hq + h;
+                else if (p.lse_layout == 2) li = (int64_t)tok * p.Hq + h;
+                else li = (int64_t)h * p.lse_hs + tok;
                 p.lse[li] = lse;
             }
         }

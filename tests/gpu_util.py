@@ -17,6 +17,23 @@ import synth
 O_ATOL = 1e-2
 O_RTOL = 1e-2
 LSE_ATOL = 1e-3
+LOG2E = 1.4426950408889634
+
+
+def lse_base(lse_layout):
+    """The layout part of an lse_layout value (without the base-2 flag)."""
+    return lse_layout & ~rsd.ATTN_LSE_LOG2
+
+
+def lse_alloc(lse_layout, B, max_sq, Tq, Hq, fill, dev):
+    base = lse_base(lse_layout)
+    if base == rsd.ATTN_LSE_PADDED_BSH:
+        shape = (B, max_sq, Hq)
+    elif base == rsd.ATTN_LSE_PACKED_TH:
+        shape = (Tq, Hq)
+    else:
+        shape = (Hq, Tq)
+    return torch.full(shape, fill, dtype=torch.float32, device=dev)
 
 
 def assert_o_close(o_gpu, o_ref, where=""):
@@ -29,7 +46,7 @@ def assert_o_close(o_gpu, o_ref, where=""):
     return float(err.max())
 
 
-def assert_lse_close(lse_gpu, lse_ref, where=""):
+def assert_lse_close(lse_gpu, lse_ref, where="", atol=LSE_ATOL):
     lg = np.asarray(lse_gpu.detach().cpu().numpy() if torch.is_tensor(lse_gpu) else lse_gpu,
                     dtype=np.float64).reshape(lse_ref.shape)
     ninf = lse_ref == -np.inf
@@ -37,7 +54,7 @@ def assert_lse_close(lse_gpu, lse_ref, where=""):
     fin = ~ninf
     assert np.all(np.isfinite(lg[fin])), f"{where}: non-finite LSE"
     err = np.abs(lg[fin] - lse_ref[fin]) if fin.any() else np.zeros(1)
-    assert err.max() <= LSE_ATOL, f"{where}: LSE max abs err {err.max():.3e}"
+    assert err.max() <= atol, f"{where}: LSE max abs err {err.max():.3e}"
     return float(err.max())
 
 
@@ -56,11 +73,8 @@ def ragged_gpu(q, k, v, cu_q, cu_kv, max_sq, max_skv, scale, causal, lse_layout=
     B = len(cu_q) - 1
     Tq = q.shape[0]
     o = torch.full((Tq, q.shape[1], v.shape[2]), o_fill, dtype=torch.bfloat16, device=dev)
-    if lse_layout == rsd.ATTN_LSE_PADDED_BSH:
-        lse = torch.full((B, max_sq, q.shape[1]), lse_fill, dtype=torch.float32, device=dev)
-    else:
-        lse = torch.full((Tq, q.shape[1]), lse_fill, dtype=torch.float32, device=dev)
     tq = Tq if total_q is None else total_q
+    lse = lse_alloc(lse_layout, B, max_sq, tq, q.shape[1], lse_fill, dev)
     ws = torch.empty(rsd.attn_fwd_ragged_workspace_size(B, max_sq, tq, q.shape[1], k.shape[1]),
                      dtype=torch.uint8, device=dev)
     cq = torch.as_tensor(np.asarray(cu_q, dtype=np.int32), device=dev)
@@ -88,11 +102,14 @@ def gather_ragged(o, lse, cu_q, rows, lse_layout=rsd.ATTN_LSE_PADDED_BSH):
     t_tok = torch.as_tensor(tok, device=o.device)
     t_h = torch.as_tensor(rows[:, 1].astype(np.int64), device=o.device)
     og = o[t_tok, t_h]
-    if lse_layout == rsd.ATTN_LSE_PADDED_BSH:
+    base = lse_base(lse_layout)
+    if base == rsd.ATTN_LSE_PADDED_BSH:
         lg = lse[torch.as_tensor(rows[:, 0].astype(np.int64), device=o.device),
                  torch.as_tensor(rows[:, 2].astype(np.int64), device=o.device), t_h]
-    else:
+    elif base == rsd.ATTN_LSE_PACKED_TH:
         lg = lse[t_tok, t_h]
+    else:
+        lg = lse[t_h, t_tok]
     return og, lg
 
 
@@ -106,9 +123,14 @@ def check_ragged(q, k, v, cu_q, cu_kv, scale, causal, rows=None, where="", **kw)
         rows = ragged_rows_all(cu_q, q.shape[1])
     o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(k), bits(v), cu_q, cu_kv, q.shape[1], k.shape[1],
                                           scale, causal, rows)
-    og, lg = gather_ragged(o, lse, cu_q, rows, kw.get("lse_layout", rsd.ATTN_LSE_PADDED_BSH))
+    layout = kw.get("lse_layout", rsd.ATTN_LSE_PADDED_BSH)
+    og, lg = gather_ragged(o, lse, cu_q, rows, layout)
     e_o = assert_o_close(og, o_ref, where)
-    e_l = assert_lse_close(lg, l_ref, where)
+    if layout & rsd.ATTN_LSE_LOG2:
+        # base-2 LSE = natural LSE * log2(e); the tolerance scales with it
+        e_l = assert_lse_close(lg, l_ref * LOG2E, where, atol=LSE_ATOL * LOG2E)
+    else:
+        e_l = assert_lse_close(lg, l_ref, where)
     return o, lse, (e_o, e_l)
 
 

@@ -94,10 +94,45 @@ def test_ragged_requires_workspace(lib):
     rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
            s2, s2, s2, s2, 0, 0.125, 1, ctypes.c_void_p(0x100100), 8, None)
     assert rc == rsd.ATTN_ERR_WORKSPACE
-    # bad LSE layout code
-    rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
-           s2, s2, s2, s2, 7, 0.125, 1, None, 0, None)
-    assert rc == rsd.ATTN_ERR_INVALID_ARG
+    # bad LSE layout codes; the valid ones (any base layout, with or without the
+    # base-2 flag) get as far as the workspace check
+    for bad in (7, 3, rsd.ATTN_LSE_LOG2 | 3, 0x200):
+        rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
+               s2, s2, s2, s2, bad, 0.125, 1, None, 0, None)
+        assert rc == rsd.ATTN_ERR_INVALID_ARG, bad
+    for good in (rsd.ATTN_LSE_PADDED_BSH, rsd.ATTN_LSE_PACKED_TH, rsd.ATTN_LSE_PACKED_HT):
+        for flag in (0, rsd.ATTN_LSE_LOG2):
+            rc = f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, 101, 4, 1, 64, 64,
+                   s2, s2, s2, s2, good | flag, 0.125, 1, None, 0, None)
+            assert rc == rsd.ATTN_ERR_WORKSPACE, (good, flag)
+
+
+def test_kv_table_entry_points_validate_both_tables(lib):
+    """The independent-table calls check the V table like the K table: a null
+    V table or a V row shorter than max_kv_len pages is rejected on the host."""
+    fake = ctypes.c_void_p(0x100000)
+    q2 = L2(64 * 128, 128)
+    kp = L3(8 * 64 * 128, 128, 64 * 128)
+    f = lib.attn_fwd_paged_kv_tables
+
+    def dec(vt, vstride):
+        return f(fake, fake, fake, fake, None, fake, 64, vt, vstride, fake, 4, 64, 8, 128, 128, 64, 100, 4096,
+                 q2, q2, kp, kp, 0.088, 3, None, 0, None)
+
+    assert dec(fake, 64) == rsd.ATTN_ERR_WORKSPACE        # both tables fine: next check is the workspace
+    assert dec(None, 64) == rsd.ATTN_ERR_INVALID_ARG
+    assert dec(fake, 63) == rsd.ATTN_ERR_INVALID_ARG      # 63 pages < 4096 / 64
+    g = lib.attn_fwd_paged_prefill_kv_tables
+    q3 = L2(32 * 128, 128)
+    kp3 = L3(4 * 64 * 128, 128, 64 * 128)
+
+    def pre(vt, vstride):
+        return g(fake, fake, fake, fake, None, fake, fake, 64, vt, vstride, fake, 2, 512, 600, 32, 4, 128, 64,
+                 100, 4096, q3, q3, kp3, kp3, rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, None, 0, None)
+
+    assert pre(fake, 64) == rsd.ATTN_ERR_WORKSPACE
+    assert pre(None, 64) == rsd.ATTN_ERR_INVALID_ARG
+    assert pre(fake, 10) == rsd.ATTN_ERR_INVALID_ARG
 
 
 def test_paged_rejects_bad_args_on_host(lib):

@@ -1,10 +1,12 @@
 """Paged decode (GQA and absorbed MLA) with split-KV on the GPU vs the fp64
 oracle, plus paged == contiguous (bit-exact), split == unsplit, NaN in the
-unused tail of the last page, and the standalone LSE merge."""
+unused tail of the last page, independent K and V page tables, and the
+standalone LSE merge."""
 import numpy as np
 import pytest
 import torch
 
+import gpu_util
 import oracle
 import ragged_scaled_dot_b200 as rsd
 import synth
@@ -224,3 +226,69 @@ def test_split_merge_kernel_vs_oracle(Dv):
     torch.cuda.synchronize()
     assert_o_close(o, o_ref, "merge")
     assert_lse_close(lse, l_ref, "merge")
+
+
+# ------------------------------------------------ independent K and V tables
+def _independent_v(v_pool, table_k, lens, ps, seed, layout="HND"):
+    """A second V pool that holds the same logical value rows as v_pool (read
+    through table_k), laid out by its own page permutation table_v.  Pages no
+    table entry names are NaN, so a read outside the table would show."""
+    lens = np.asarray(lens, dtype=np.int64)
+    n_pages = (lens + ps - 1) // ps
+    table_v, total = synth.page_table(lens, ps, seed)
+    v2 = torch.full((total + 5,) + tuple(v_pool.shape[1:]), float("nan"), dtype=v_pool.dtype, device=DEV)
+    src = np.concatenate([table_k[b, :n] for b, n in enumerate(n_pages)] + [np.zeros(0, np.int32)])
+    dst = np.concatenate([table_v[b, :n] for b, n in enumerate(n_pages)] + [np.zeros(0, np.int32)])
+    v2[torch.as_tensor(dst.astype(np.int64), device=DEV)] = v_pool[torch.as_tensor(src.astype(np.int64),
+                                                                                    device=DEV)]
+    return v2, table_v
+
+
+def _paged_kv_tables_gpu(q, k_pool, v_pool, table_k, table_v, kl, ps, scale, splits, Dv, layout="HND"):
+    B, Hq, _ = q.shape
+    o = torch.full((B, Hq, Dv), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=DEV)
+    ws_n = rsd.attn_fwd_paged_workspace_size(B, Hq, Dv, splits)
+    ws = torch.full((ws_n,), 0xFF, dtype=torch.uint8, device=DEV) if ws_n else None
+    rsd.attn_fwd_paged_kv_tables(q, k_pool, v_pool, o, lse, torch.as_tensor(table_k, device=DEV),
+                                 torch.as_tensor(table_v, device=DEV), torch.as_tensor(kl, device=DEV),
+                                 page_size=ps, max_kv_len=max(1, int(np.max(kl))), scale=scale,
+                                 num_splits=splits, workspace=ws, kv_layout=layout)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,ps,layout,splits", [
+    ([0, 1, 700, 130], 16, 2, 128, 64, "HND", 1),
+    ([0, 1, 700, 130], 16, 2, 128, 64, "HND", 3),
+    ([300, 45], 8, 1, 64, 16, "NHD", 2),
+])
+def test_gqa_decode_independent_kv_tables(lens, Hq, Hkv, D, ps, layout, splits):
+    """K through one page table, V through another over a different pool: the
+    oracle's result for the same logical K/V, and bit-identical to one shared
+    table over a pool that stores V where K's table points."""
+    q, k, v, table, kl = _paged_inputs(lens, Hq, Hkv, D, ps, seed=53 + ps, layout=layout)
+    v2, table_v = _independent_v(v, table, lens, ps, seed=59 + ps, layout=layout)
+    assert not np.array_equal(table, table_v)
+    o, lse = _paged_kv_tables_gpu(q, k, v2, table, table_v, kl, ps, 1.0 / np.sqrt(D), splits, D, layout)
+    o1, l1 = paged_gpu(q, k, v, table, kl, ps, 1.0 / np.sqrt(D), splits, kv_layout=layout)
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    rows = np.array([(b, h) for b in range(len(lens)) for h in range(Hq)], dtype=np.int32)
+    o_ref, l_ref = orc().attn_paged_rows(bits(q), bits(k), bits(v), table, kl, ps, Hq, Hkv, D, D,
+                                         gpu_util.pool_strides_np(k, layout), gpu_util.pool_strides_np(v, layout),
+                                         1.0 / np.sqrt(D), rows)
+    assert_o_close(o.reshape(-1, D), o_ref, "independent tables")
+    assert_lse_close(lse.reshape(-1), l_ref, "independent tables")
+
+
+@pytest.mark.parametrize("splits", [1, 2])
+def test_mla_decode_independent_kv_tables(splits):
+    """Absorbed-MLA shapes (Q/K 576, V 512) with V in its own pool and page table."""
+    lens, ps = [100, 700, 64], 64
+    q, k, v, table, kl = _paged_inputs(lens, 128, 1, 576, ps, seed=61, Dv=512)
+    v2, table_v = _independent_v(v, table, lens, ps, seed=67)
+    o, lse = _paged_kv_tables_gpu(q, k, v2, table, table_v, kl, ps, 1.0 / np.sqrt(576), splits, 512)
+    o1, l1 = paged_gpu(q, k, v, table, kl, ps, 1.0 / np.sqrt(576), splits, o_dv=512)
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(576), splits, Dv=512, where="mla independent tables")

@@ -10,7 +10,8 @@ import torch
 
 import ragged_scaled_dot_b200 as rsd
 import synth
-from gpu_util import assert_lse_close, assert_o_close, bits, gather_ragged, orc, ragged_gpu, ragged_rows_all
+from gpu_util import (LOG2E, LSE_ATOL, assert_lse_close, assert_o_close, bits, gather_ragged, lse_alloc, orc,
+                      ragged_gpu, ragged_rows_all)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -46,10 +47,7 @@ def _run(q, k, v, table, kl, cu_q, ps, scale, causal, layout="HND", lse_layout=r
     max_sq = max(1, int(np.max(np.diff(cu_q))))
     Hq = q.shape[1]
     o = torch.full((q.shape[0], Hq, v.shape[-1]), float("nan"), dtype=torch.bfloat16, device=DEV)
-    if lse_layout == rsd.ATTN_LSE_PADDED_BSH:
-        lse = torch.full((B, max_sq, Hq), float("nan"), dtype=torch.float32, device=DEV)
-    else:
-        lse = torch.full((q.shape[0], Hq), float("nan"), dtype=torch.float32, device=DEV)
+    lse = lse_alloc(lse_layout, B, max_sq, q.shape[0], Hq, float("nan"), DEV)
     Hkv = k.shape[1] if layout == "HND" else k.shape[2]
     ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(B, max_sq, q.shape[0], Hq, Hkv),
                      dtype=torch.uint8, device=DEV)
@@ -113,3 +111,53 @@ def test_paged_prefill_nan_past_kv_len_is_never_used(ps):
     o2, l2 = _run(q, kn, vn, table, kl, cu_q, ps, 0.1, True)
     assert torch.isfinite(o2.float()).all()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_paged_prefill_head_major_base2_lse():
+    """Head-major [Hq, total_q] LSE in base 2 (stats_use_log2) over a paged
+    cache: the oracle's natural LSE times log2(e)."""
+    lens_q, lens_kv, ps = [3, 130, 1], [700, 130, 64], 64
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=21)
+    lay = rsd.ATTN_LSE_PACKED_HT | rsd.ATTN_LSE_LOG2
+    o, lse = _run(q, k, v, table, kl, cu_q, ps, 0.09, True, lse_layout=lay)
+    kc, vc = _gather(k, table, kl, ps, "HND"), _gather(v, table, kl, ps, "HND")
+    cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
+    rows = ragged_rows_all(cu_q, 8)
+    o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(kc), bits(vc), cu_q, cu_kv, 8, 2, 0.09, True, rows)
+    og, lg = gather_ragged(o, lse, cu_q, rows, lay)
+    assert_o_close(og, o_ref, "paged prefill, head-major base-2 LSE")
+    assert_lse_close(lg, l_ref * LOG2E, "paged prefill, head-major base-2 LSE", atol=LSE_ATOL * LOG2E)
+
+
+def test_paged_prefill_independent_kv_tables():
+    """Chunked prefill with V in its own pool and page table: the oracle's
+    result, and bit-identical to one shared table over the original pool."""
+    lens_q, lens_kv, ps = [3, 130, 64], [700, 130, 300], 64
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=71)
+    n_pages = [(L + ps - 1) // ps for L in lens_kv]
+    table_v, total = synth.page_table(lens_kv, ps, 73)
+    v2 = torch.full((total + 4,) + tuple(v.shape[1:]), float("nan"), dtype=v.dtype, device=DEV)
+    src = np.concatenate([table[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
+    dst = np.concatenate([table_v[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
+    v2[torch.as_tensor(dst, device=DEV)] = v[torch.as_tensor(src, device=DEV)]
+    B, Hq = len(lens_q), 8
+    o = torch.full((q.shape[0], Hq, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = lse_alloc(rsd.ATTN_LSE_PACKED_TH, B, max(lens_q), q.shape[0], Hq, float("nan"), DEV)
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(B, max(lens_q), q.shape[0], Hq, 2),
+                     dtype=torch.uint8, device=DEV)
+    rsd.attn_fwd_paged_prefill_kv_tables(
+        q, k, v2, o, lse, torch.as_tensor(cu_q, device=DEV), torch.as_tensor(table, device=DEV),
+        torch.as_tensor(table_v, device=DEV), torch.as_tensor(kl, device=DEV), max_seqlen_q=max(lens_q),
+        page_size=ps, max_kv_len=max(lens_kv), scale=0.09, causal=True, workspace=ws,
+        lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    o1, l1 = _run(q, k, v, table, kl, cu_q, ps, 0.09, True, lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    kc, vc = _gather(k, table, kl, ps, "HND"), _gather(v, table, kl, ps, "HND")
+    cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
+    rows = ragged_rows_all(cu_q, Hq)
+    o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(kc), bits(vc), cu_q, cu_kv, Hq, 2, 0.09, True, rows)
+    og, lg = gather_ragged(o, lse, cu_q, rows, rsd.ATTN_LSE_PACKED_TH)
+    assert_o_close(og, o_ref, "paged prefill, independent tables")
+    assert_lse_close(lg, l_ref, "paged prefill, independent tables")

@@ -1,14 +1,15 @@
 """Prefill (dense BSHD and ragged THD) on the GPU vs the fp64 oracle, plus the
 invariants that pin the kernel: causality, determinism, ragged == dense,
-GQA == replicated MHA, strided views, NaN tails, padded LSE rows."""
+GQA == replicated MHA, strided and gapped views, NaN tails, every LSE layout
+in both bases."""
 import numpy as np
 import pytest
 import torch
 
 import ragged_scaled_dot_b200 as rsd
 import synth
-from gpu_util import (assert_lse_close, assert_o_close, bits, check_dense, check_ragged,
-                      dense_gpu, orc, ragged_gpu, ragged_rows_all)
+from gpu_util import (LOG2E, assert_lse_close, assert_o_close, bits, check_dense, check_ragged,
+                      dense_gpu, gather_ragged, orc, ragged_gpu, ragged_rows_all)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -59,6 +60,62 @@ def test_ragged_packed_lse_layout():
     q, k, v, cu_q, cu_kv = _ragged_inputs(lq, lq, 4, 2, 128, seed=5)
     check_ragged(q, k, v, cu_q, cu_kv, 0.1, True, lse_layout=rsd.ATTN_LSE_PACKED_TH,
                  where="packed LSE")
+
+
+@pytest.mark.parametrize("layout", ["PADDED_BSH", "PACKED_TH", "PACKED_HT"])
+@pytest.mark.parametrize("log2", [False, True])
+def test_ragged_lse_layouts_and_base(layout, log2):
+    """Every LSE layout (padded per batch, token-major, head-major [Hq, total_q])
+    in natural log and in base 2 (stats_use_log2): base 2 is the natural LSE
+    times log2(e), -inf rows stay -inf, padded rows past a sequence stay -inf."""
+    lq, lkv = [100, 3, 260, 0, 40], [100, 500, 260, 7, 0]
+    q, k, v, cu_q, cu_kv = _ragged_inputs(lq, lkv, 4, 2, 128, seed=9)
+    flag = rsd.ATTN_LSE_LOG2 if log2 else 0
+    lay = getattr(rsd, "ATTN_LSE_" + layout) | flag
+    o, lse, _ = check_ragged(q, k, v, cu_q, cu_kv, 0.1, True, lse_layout=lay, where=f"LSE {layout} log2={log2}")
+    if layout == "PADDED_BSH":
+        for b, L in enumerate(lq):
+            assert torch.all(lse[b, L:] == -float("inf"))
+    # the same call in the other base: same O bits, LSE related by log2(e) up to fp32 rounding
+    o2, lse2 = ragged_gpu(q, k, v, cu_q, cu_kv, max(lq), max(lkv), 0.1, True,
+                          lse_layout=getattr(rsd, "ATTN_LSE_" + layout) | (flag ^ rsd.ATTN_LSE_LOG2))
+    assert torch.equal(o, o2)
+    nat, b2 = (lse2, lse) if log2 else (lse, lse2)
+    fin = torch.isfinite(nat)
+    assert torch.equal(fin, torch.isfinite(b2)) and torch.all(b2[~fin] == nat[~fin])
+    assert torch.allclose(b2[fin].double(), nat[fin].double() * LOG2E, rtol=2e-6, atol=2e-6)
+
+
+def test_ragged_gapped_token_and_head_strides():
+    """Q, K, V and O as views with gaps on both THD axes (token stride larger
+    than heads x D, head stride larger than D, a nonzero base offset) are read
+    and written in place; the gaps are never touched."""
+    lq, lkv = [130, 5, 257], [200, 5, 257]
+    Hq, Hkv, D = 4, 2, 128
+    cu_q = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    cu_kv = np.concatenate([[0], np.cumsum(lkv)]).astype(np.int32)
+    Tq, Tk = int(cu_q[-1]), int(cu_kv[-1])
+    qb = synth.normal_bf16((Tq, Hq + 3, D), 31, "cpu").to(DEV)
+    kb = synth.normal_bf16((Tk, 2 * Hkv, D), 32, "cpu").to(DEV)
+    vb = synth.normal_bf16((Tk, Hkv, 2 * D), 33, "cpu").to(DEV)
+    q = qb[:, 1:Hq + 1, :]              # token gap 3 heads, base offset one head
+    k = kb[:, ::2, :]                   # head stride 2 D
+    v = vb[:, :, D:]                    # head stride 2 D, base offset D
+    ob = torch.full((Tq, Hq, 2 * D), 7.0, dtype=torch.bfloat16, device=DEV)
+    o = ob[:, :, :D]
+    lse = torch.full((len(lq), max(lq), Hq), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.empty(rsd.attn_fwd_ragged_workspace_size(len(lq), max(lq), Tq, Hq, Hkv), dtype=torch.uint8,
+                     device=DEV)
+    rsd.attn_fwd_ragged(q, k, v, o, lse, torch.as_tensor(cu_q, device=DEV), torch.as_tensor(cu_kv, device=DEV),
+                        max_seqlen_q=max(lq), max_seqlen_kv=max(lkv), scale=0.1, causal=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    assert torch.all(ob[:, :, D:] == 7.0)  # the gaps of O are left alone
+    rows = ragged_rows_all(cu_q, Hq)
+    o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(k), bits(v), cu_q, cu_kv, Hq, Hkv, 0.1, True, rows)
+    og, lg = gather_ragged(o, lse, cu_q, rows)
+    assert_o_close(og, o_ref, "gapped strides")
+    assert_lse_close(lg, l_ref, "gapped strides")
 
 
 def test_ragged_scale_zero_and_negative():
