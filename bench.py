@@ -37,12 +37,14 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill attention TFLOPS and paged-decode KV GB/s, % of B200 roofline"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes (read + write) from the latest ncu capture of each kernel
-# (profiles/), as a ratio to the bytes that scale with the launch, applied to
+# DRAM bytes (read + write) from the latest ncu capture of each kernel on its
+# small case, as a ratio to the bytes that scale with the launch, applied to
 # the full launch.  None when the kernel changed after the counters were taken.
-#   paged_decode: per K/V byte, profiles/decode_gqa_kernel_paged_b32.md (2.692 / 2.673 GB)
-#   ragged_prefill: per Q+K+V+O byte, profiles/prefill_kernel_ragged_b16.md (1.045 / 1.061 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.984, "paged_decode": 1.0071}
+#   paged_decode: per K/V byte, batch 32 (2.692 / 2.673 GB)
+#   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.041 / 1.061 GB)
+#   mla_decode: per K/V byte, batch 8 (0.345 / 0.335 GB; the partials grow with the
+#     batch like the K/V bytes)
+TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0069, "mla_decode": 1.0271}
 
 
 def load_peaks():
