@@ -40,11 +40,11 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) from the latest ncu capture of each kernel on its
 # small case, as a ratio to the bytes that scale with the launch, applied to
 # the full launch.  None when the kernel changed after the counters were taken.
-#   paged_decode: per K/V byte, batch 32 (2.692 / 2.673 GB)
+#   paged_decode: per K/V byte, batch 32 (2.686 / 2.673 GB)
 #   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.041 / 1.061 GB)
-#   mla_decode: per K/V byte, batch 8 (0.345 / 0.335 GB; the partials grow with the
+#   mla_decode: per K/V byte, batch 8 (0.346 / 0.335 GB; the partials grow with the
 #     batch like the K/V bytes)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0069, "mla_decode": 1.0271}
+TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307}
 
 
 def load_peaks():
@@ -288,7 +288,7 @@ def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
             "flop_per_step": flops, "total_pages": int(kp.shape[0]),
             "bytes_per_unit": f"{w.Hkv * (w.Dqk if w.v_aliases_k else w.Dqk + Dv) * 2} B of K/V per cached token"}
     data = dict(q=q, kp=kp, vp=vp, table=table, L=L, w=w, S=S)
-    launches = 2 if S > 1 else 1
+    launches = 3 if S > 1 else 1  # with splits: the launch-order sort, the decode, the merge
     return Part(name, "GB/s", nbytes / 1e9, launches, step, e2e_setup, info), data
 
 

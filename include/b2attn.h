@@ -200,8 +200,10 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  * Split-KV: each sequence's pages are cut into num_splits ranges of
  * ceil(n_pages / num_splits) consecutive pages; num_splits > 1 writes fp32
  * partial O and LSE into the workspace and merges them as attn_split_merge
- * does.  workspace: >= attn_fwd_paged_workspace_size(...) bytes, 256-byte
- * aligned (may be NULL when num_splits == 1).
+ * does, and the blocks take the sequences longest first (a device-side sort
+ * of kv_lens into the workspace; it changes which block computes a split,
+ * never the result).  workspace: >= attn_fwd_paged_workspace_size(...) bytes,
+ * 256-byte aligned (may be NULL when num_splits == 1).
  */
 int attn_fwd_paged(const void *q, const void *k_pool, const void *v_pool, void *o,
                    float *lse, const int32_t *page_table, int64_t page_table_stride,

@@ -540,7 +540,9 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits) {
     if (B <= 0 || Hq <= 0 || Dv <= 0 || num_splits <= 1) return 0;
     const int64_t R = (int64_t)B * Hq;
-    return (size_t)(round_up(R * num_splits * Dv * 4, 256) + round_up(R * num_splits * 4, 256));
+    // partial O, partial LSE, launch order of the sequences
+    return (size_t)(round_up(R * num_splits * Dv * 4, 256) + round_up(R * num_splits * 4, 256) +
+                    round_up((int64_t)B * 4, 256));
 }
 
 int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len, int page_size,
@@ -550,16 +552,20 @@ int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_k
     int64_t s_balance;
     double max_overhead;
     if (mla) {
-        // a cluster of two CTAs (one per SM) per (sequence, split, 128-head group): about five
-        // waves of work units over the SM pairs, partial traffic up to ~10% of the KV bytes
+        // a cluster of two CTAs (one per SM) per (sequence, split, 128-head group): about three
+        // waves of work units over the SM pairs (the launch order puts the longest sequences
+        // first, so few waves suffice; measured best on the 64-sequence MLA workload against
+        // 1, 2, 4 and 5), partial traffic up to ~10% of the KV bytes
         const int64_t units_per_split = (int64_t)B * ((Hq + 127) / 128);
         const int64_t pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
-        s_balance = (5 * pairs + units_per_split - 1) / units_per_split;
+        s_balance = (3 * pairs + units_per_split - 1) / units_per_split;
         max_overhead = 0.10;
     } else {
         const int64_t ctas_per_split = (int64_t)Hkv * B;
         const int64_t slots = (int64_t)num_sms * 2;
-        s_balance = (8 * slots + ctas_per_split - 1) / ctas_per_split;
+        // about four waves of CTAs over the two resident CTAs per SM (longest sequences
+        // first; measured best on the 128-sequence GQA workload against 8 and 16)
+        s_balance = (4 * slots + ctas_per_split - 1) / ctas_per_split;
         max_overhead = 0.05;
     }
     // the fp32 partials (written + read) stay under max_overhead of the KV bytes streamed
@@ -674,9 +680,17 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     dp.lse = lse;
     const int64_t R = (int64_t)B * Hq;
     if (num_splits > 1) {
-        dp.o_part = static_cast<float*>(workspace);
-        dp.lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
-                                               round_up(R * num_splits * Dv * 4, 256));
+        char* wsb = static_cast<char*>(workspace);
+        dp.o_part = reinterpret_cast<float*>(wsb);
+        dp.lse_part = reinterpret_cast<float*>(wsb + round_up(R * num_splits * Dv * 4, 256));
+        // sequences longest first: the blocks of the longest splits start first
+        int32_t* order = reinterpret_cast<int32_t*>(wsb + round_up(R * num_splits * Dv * 4, 256) +
+                                                    round_up(R * num_splits * 4, 256));
+        int shift = 0;
+        while ((max_kv_len >> shift) >= 4096) ++shift;
+        b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order);
+        if (int e = launch_status()) return e;
+        dp.order = order;
     }
     if (mla) {
         // one cluster of two CTAs (score CTA, value CTA) per (b, split, group of 128 heads)

@@ -13,7 +13,9 @@
 // [s*pps, min((s+1)*pps, n_pages)), pps = ceil(n_pages / num_splits).
 // With one split the kernel writes O (bf16) and LSE directly; otherwise it
 // writes the normalised fp32 partial O_s and its natural-log lse_s, and
-// split_merge_kernel combines them.
+// split_merge_kernel combines them.  With splits, blocks take the sequences in
+// the order seq_order_kernel leaves in the workspace (longest first), so the
+// longest splits start first and the short ones fill the tail.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,6 +32,7 @@ struct DecodeParams {
     const int32_t* v_page_table;  // V pages (the K table unless the caller gives its own)
     int64_t v_pt_stride;
     const int32_t* kv_lens;
+    const int32_t* order;  // launch order (sequences longest first) or null: block z runs sequence order[z]
     int B, Hq, Hkv, G;
     int page_size, box_rows;  // rows per TMA box: min(page_size, chunk keys)
     int64_t num_pages;
@@ -119,7 +122,8 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
     auto empty_bar = [&](int i) { return sBar + 8u * (NST + i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + C::BAR_OFF + 16u * NST);
 
-    const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int s = blockIdx.x, g = blockIdx.y;
+    const int b = p.order ? __ldg(p.order + blockIdx.z) : (int)blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int L, lo, hi;
     decode_split_range(p, b, s, L, lo, hi);

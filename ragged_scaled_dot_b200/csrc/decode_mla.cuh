@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
     const int hg = unit % n_hg;
     const int bs = unit / n_hg;
     const int s = bs % p.num_splits;
-    const int b = bs / p.num_splits;
+    const int b = p.order ? __ldg(p.order + bs / p.num_splits) : bs / p.num_splits;
     const int nh = min(128, p.Hq - hg * 128);
     int L, lo, hi;
     decode_split_range(p, b, s, L, lo, hi);

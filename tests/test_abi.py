@@ -197,3 +197,24 @@ def test_paged_prefill_rejects_bad_args_on_host(lib):
     assert call(B=0) == rsd.ATTN_OK                          # nothing to do
     assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 32, 4) == \
         rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 32, 4)
+
+
+def test_sizes_past_the_32_bit_token_range_are_declined(lib):
+    """Token counts of 2^31 or more (32-bit token coordinates of the tensor
+    maps and the work list) and grids past the launch limits are declined
+    with ATTN_ERR_UNSUPPORTED on the host, never computed wrongly."""
+    fake = ctypes.c_void_p(0x100000)
+    s2 = L2(4 * 64, 64)
+    big = 1 << 31
+    f = lib.attn_fwd_ragged
+    assert f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, big, 101, 4, 1, 64, 64,
+             s2, s2, s2, s2, 0, 0.125, 1, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED
+    assert f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, 101, big, 4, 1, 64, 64,
+             s2, s2, s2, s2, 0, 0.125, 1, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED
+    assert f(fake, fake, fake, fake, None, fake, fake, 2, 64, 64, big - 1, 101, 4, 1, 64, 64,
+             s2, s2, s2, s2, 0, 0.125, 1, None, 0, None) == rsd.ATTN_ERR_WORKSPACE
+    g = lib.attn_fwd_paged
+    q2 = L2(64 * 128, 128)
+    kp = L3(8 * 64 * 128, 128, 64 * 128)
+    assert g(fake, fake, fake, fake, None, fake, 64, fake, 65536, 64, 8, 128, 128, 64, 100, 4096,
+             q2, q2, kp, kp, 0.088, 1, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED   # B > 65535

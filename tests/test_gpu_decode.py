@@ -292,3 +292,23 @@ def test_mla_decode_independent_kv_tables(splits):
     o1, l1 = paged_gpu(q, k, v, table, kl, ps, 1.0 / np.sqrt(576), splits, o_dv=512)
     assert torch.equal(o, o1) and torch.equal(lse, l1)
     check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(576), splits, Dv=512, where="mla independent tables")
+
+
+@pytest.mark.parametrize("mla", [False, True])
+def test_decode_batch_permutation_bitwise(mla):
+    """With splits the blocks take the sequences longest first (a device-side
+    sort of kv_lens): permuting the batch permutes the outputs bit for bit, so
+    every split lands on its own sequence whatever block runs it."""
+    lens = [3000, 10, 700, 700, 1, 2049, 64]
+    if mla:
+        q, k, v, table, kl = _paged_inputs(lens, 128, 1, 576, 64, seed=79, Dv=512)
+        Dv, S = 512, 4
+    else:
+        q, k, v, table, kl = _paged_inputs(lens, 16, 2, 128, 64, seed=83)
+        Dv, S = 128, 3
+    o1, l1 = paged_gpu(q, k, v, table, kl, 64, 0.07, S, o_dv=Dv)
+    perm = np.array([4, 0, 6, 2, 5, 3, 1])
+    o2, l2 = paged_gpu(q[torch.as_tensor(perm, device=DEV)].contiguous(), k, v, table[perm], kl[perm], 64, 0.07, S,
+                       o_dv=Dv)
+    assert torch.equal(o2, o1[torch.as_tensor(perm, device=DEV)])
+    assert torch.equal(l2, l1[torch.as_tensor(perm, device=DEV)])
