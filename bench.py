@@ -81,16 +81,39 @@ def decode_kv_bytes(kv_lens, Hkv, Dqk, Dv, alias):
 # clocks sampler
 # --------------------------------------------------------------------------- #
 class ClockSampler:
+    """SM clock, its maximum and the clock-event reasons, sampled while the
+    parts are timed: read-only NVML queries every 20 ms from a thread (the GPU
+    matched by PCI bus id, which holds under CUDA_VISIBLE_DEVICES), else
+    `nvidia-smi -lms 100`.  Lines are kept in nvidia-smi's CSV field order."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits (nvml.h): hw_slowdown, hw_thermal_slowdown,
+    # sw_thermal_slowdown, sw_power_cap, in FIELDS order
+    REASON_BITS = (0x8, 0x40, 0x20, 0x4)
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.nvml = None
         self.lines = []
 
     def __enter__(self):
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(self.index)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nvml = pynvml
+            self._stop = threading.Event()
+            self._sample_nvml()  # one sample before the timing starts
+            self._t = threading.Thread(target=self._loop_nvml, daemon=True)
+            self._t.start()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
@@ -102,11 +125,34 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def _sample_nvml(self):
+        n, h = self.nvml, self.handle
+        sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+        watts = n.nvmlDeviceGetPowerUsage(h) / 1000.0
+        r = n.nvmlDeviceGetCurrentClocksEventReasons(h)
+        flags = ["Active" if r & bit else "Not Active" for bit in self.REASON_BITS]
+        self.lines.append(", ".join([str(sm), str(mx), f"{watts:.1f}", hex(r)] + flags))
+
+    def _loop_nvml(self):
+        while not self._stop.wait(0.02):
+            try:
+                self._sample_nvml()
+            except Exception:
+                return
+
     def _read(self):
         for ln in self.proc.stdout:
             self.lines.append(ln.strip())
 
     def __exit__(self, *a):
+        if self.nvml is not None:
+            self._stop.set()
+            self._t.join(timeout=5)
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
