@@ -180,7 +180,9 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  * its kv_lens[b] cached keys ("cuDNN Frontend v1.31.0 Release Notes", "SDPA:
  * paged KV, split-KV, and engine selection").
  *   q: [B, Hq, Dqk] with (batch, head) element strides q_strides[2].
- *   o: [B, Hq, Dv]  with (batch, head) element strides o_strides[2].
+ *   o: [B, Hq, Dv]  with (batch, head) element strides o_strides[2]; with
+ *   num_splits > 1 the rows must be batch-major (o_strides[0] == Hq *
+ *   o_strides[1]), else ATTN_ERR_UNSUPPORTED before anything is enqueued.
  *   lse (nullable): fp32 [B, Hq] contiguous.
  *   k_pool / v_pool: pools of num_pages fixed-size pages; element
  *   (page, slot, head, d) at pool[page*s[0] + slot*s[1] + head*s[2] + d] with

@@ -625,6 +625,8 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     for (int i = 0; i < 3; ++i)
         if (!stride_ok(k_pool_strides[i]) || !stride_ok(v_pool_strides[i])) return ATTN_ERR_INVALID_ARG;
     if (num_splits > 1) {
+        // the merge writes O row r = b*Hq + h at o + r*o_strides[1]: batch-major rows
+        if (o_strides[0] != (int64_t)Hq * o_strides[1]) return ATTN_ERR_UNSUPPORTED;
         const size_t need = attn_fwd_paged_workspace_size(B, Hq, Dv, num_splits);
         if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
@@ -718,11 +720,8 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
             b2::decode_gqa_kernel<64><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
     }
     if (int e = launch_status()) return e;
-    if (num_splits > 1) {
-        // O rows are (b, h); merge writes row r = b*Hq + h at o + b*o_bs + h*o_hs.
-        if (o_strides[0] != (int64_t)Hq * o_strides[1]) return ATTN_ERR_UNSUPPORTED;
+    if (num_splits > 1)
         return attn_split_merge(dp.o_part, dp.lse_part, num_splits, R, Dv, o, o_strides[1], lse, stream);
-    }
     return ATTN_OK;
 }
 

@@ -149,6 +149,10 @@ def test_paged_rejects_bad_args_on_host(lib):
                  None)
 
     assert call() == rsd.ATTN_ERR_WORKSPACE              # 3 splits need a workspace
+    # split outputs go through the merge, which needs batch-major O rows: refused on the
+    # host, before the workspace is even looked at
+    assert f(fake, fake, fake, fake, None, fake, 64, fake, 4, 64, 8, 128, 128, 64, 100, 4096,
+             q2, L2(64 * 128 + 8, 128), kp, kp, 0.088, 3, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED
     assert call(Dqk=96, Dv=96) == rsd.ATTN_ERR_UNSUPPORTED
     assert call(ps=48) == rsd.ATTN_ERR_UNSUPPORTED        # neither divides nor is divided by 64
     assert call(Hkv=7) == rsd.ATTN_ERR_INVALID_ARG        # 64 % 7 != 0
