@@ -44,7 +44,8 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 #   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.041 / 1.061 GB)
 #   mla_decode: per K/V byte, batch 8 (0.346 / 0.335 GB; the partials grow with the
 #     batch like the K/V bytes)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307}
+#   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.683 / 0.635 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307, "paged_prefill": 1.0764}
 
 
 def load_peaks():
@@ -278,8 +279,10 @@ def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
         rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, cud, pt, kld, max_seqlen_q=smax, page_size=w.page_size,
                                    max_kv_len=maxL, scale=w.scale, causal=True, workspace=ws)
     flops = prefill_flops(lq, L, w.Hq, w.Dqk)
+    # bytes that scale with the launch: Q and O of every query, K and V of every cached key
+    io_gb = (T * 2 * w.Hq * w.Dqk * 2 + int(L.sum()) * 2 * w.Hkv * w.Dqk * 2) / 1e9
     info = {"workload": w.notes, "flop_per_step": flops, "query_tokens": int(T),
-            "kv_tokens": int(L.sum()), "total_pages": int(kp.shape[0])}
+            "kv_tokens": int(L.sum()), "total_pages": int(kp.shape[0]), "traffic_basis_gb": io_gb}
     return Part("paged_prefill", "TFLOP/s", flops / 1e12, 3, step, None, info), None
 
 
