@@ -227,3 +227,18 @@ def test_dense_strided_views_of_fused_qkv():
     qkv = synth.normal_bf16((B, S, Hq + 2 * Hkv, D), 71, "cpu").to(DEV)
     q, k, v = qkv[:, :, :Hq], qkv[:, :, Hq:Hq + Hkv], qkv[:, :, Hq + Hkv:]
     check_dense(q, k, v, 0.1, True, where="fused qkv views")
+
+
+@pytest.mark.parametrize("scale", [0.3, -0.3])
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_running_max_jumps(scale, causal):
+    """Key rows scaled by 1 + 3 t / L along each sequence make the scores grow
+    (or, with a negative scale, fall) from tile to tile, so the running row
+    maximum moves by more than 2^8 many times: the O rescale and the recompute
+    of a tile against a new maximum both run.  V stays N(0,1)."""
+    lens = [1500, 700, 130]
+    Hq, Hkv, D = 4, 2, 128
+    q, k, v, cu_q, cu_kv = _ragged_inputs(lens, lens, Hq, Hkv, D, seed=89)
+    f = torch.cat([1.0 + 3.0 * torch.arange(L, dtype=torch.float32) / L for L in lens]).to(DEV)
+    k = (k.float() * f[:, None, None]).to(torch.bfloat16)
+    check_ragged(q, k, v, cu_q, cu_kv, scale, causal, where=f"running max jumps scale={scale} causal={causal}")
