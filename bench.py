@@ -45,7 +45,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 #   mla_decode: per K/V byte, batch 8 (0.346 / 0.335 GB; the partials grow with the
 #     batch like the K/V bytes)
 #   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.683 / 0.635 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307, "paged_prefill": 1.0764}
+#   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (1.049 / 0.671 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307, "paged_prefill": 1.0764,
+                 "dense_prefill": 1.5627}
 
 
 def load_peaks():
@@ -264,7 +266,9 @@ def make_dense_prefill(torch, rsd, synth, dev, seed_offset, B=0):
     def step():
         rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True)
     flops = prefill_flops([w.S] * w.B, [w.S] * w.B, w.Hq, w.Dqk)
-    info = {"workload": w.notes, "flop_per_step": flops}
+    # bytes that scale with the launch: Q, K, V and O
+    io_gb = w.B * w.S * (2 * w.Hq * w.Dqk + w.Hkv * (w.Dqk + w.Dv)) * 2 / 1e9
+    info = {"workload": w.notes, "flop_per_step": flops, "traffic_basis_gb": io_gb}
     return Part("dense_prefill", "TFLOP/s", flops / 1e12, 1, step, None, info), None
 
 

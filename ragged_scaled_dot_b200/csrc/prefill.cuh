@@ -109,15 +109,24 @@ __device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal)
 
 __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx, PrefillItem& it) {
     if (p.mode == 0) {
-        // dense: (query tile longest first, batch, kv head, head pair): the static
-        // round-robin assignment then hands out the longest items first
-        const int per_t = p.B * p.Hkv * p.pairs_per_group;
-        const int t = idx / per_t;
-        int rem = idx - t * per_t;
-        it.b = rem / (p.Hkv * p.pairs_per_group);
-        rem -= it.b * p.Hkv * p.pairs_per_group;
-        const int g = rem / p.pairs_per_group;
-        const int pr = rem - g * p.pairs_per_group;
+        // dense: groups of kQtGroup query tiles, the longest group first; inside a group
+        // (batch, kv head, query tile longest first, head pair).  The static round-robin
+        // assignment then hands out items of nearly equal length side by side, and the
+        // CTAs working at the same time share few (batch, kv head) K/V streams in L2.
+        constexpr int kQtGroup = 4;
+        const int per_t = p.B * p.Hkv * p.pairs_per_group;  // items per query tile
+        const int grp = idx / (kQtGroup * per_t);
+        const int t0 = grp * kQtGroup;
+        const int nt = min(kQtGroup, p.n_qtiles - t0);       // tiles in this (maybe last) group
+        int rem = idx - t0 * per_t;
+        const int per_bg = nt * p.pairs_per_group;           // items per (batch, kv head) in the group
+        const int bg = rem / per_bg;
+        rem -= bg * per_bg;
+        it.b = bg / p.Hkv;
+        const int g = bg - it.b * p.Hkv;
+        const int ti = rem / p.pairs_per_group;
+        const int pr = rem - ti * p.pairs_per_group;
+        const int t = t0 + ti;
         it.qt = p.causal ? (p.n_qtiles - 1 - t) : t;
         it.h0 = g * p.G + pr * p.heads_per_item;
         it.q_tok0 = it.qt * 128;
