@@ -262,14 +262,16 @@ def make_dense_prefill(torch, rsd, synth, dev, seed_offset, B=0):
     q, k, v = synth.make_dense(g, dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.S), dtype=torch.float32, device=dev)
+    ws = torch.empty(rsd.attn_fwd_dense_workspace_size(w.B, w.S, w.Hq, w.Hkv), dtype=torch.uint8, device=dev)
 
     def step():
-        rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True)
+        rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True, workspace=ws)
     flops = prefill_flops([w.S] * w.B, [w.S] * w.B, w.Hq, w.Dqk)
     # bytes that scale with the launch: Q, K, V and O
     io_gb = w.B * w.S * (2 * w.Hq * w.Dqk + w.Hkv * (w.Dqk + w.Dv)) * 2 / 1e9
     info = {"workload": w.notes, "flop_per_step": flops, "traffic_basis_gb": io_gb}
-    return Part("dense_prefill", "TFLOP/s", flops / 1e12, 1, step, None, info), None
+    # the device work list and the prefill kernel
+    return Part("dense_prefill", "TFLOP/s", flops / 1e12, 2, step, None, info), None
 
 
 def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):

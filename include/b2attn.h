@@ -100,13 +100,28 @@ const char *attn_status_string(int status);
  * x_strides[3] are the (batch, seq, head) element strides of each tensor, so
  * strided views (e.g. slices of a fused QKV projection) are read in place
  * ("cuDNN Frontend v1.30.0 Release Notes", "New: prepared launches": dense
- * forward reads strided Q/K/V/O zero-copy).  Needs no workspace.
+ * forward reads strided Q/K/V/O zero-copy).  With Sq != Skv the causal mask
+ * is bottom-right aligned.
+ * workspace: device scratch of at least attn_fwd_dense_workspace_size(...)
+ * bytes, 256-byte aligned, owned by the caller ("cuDNN Frontend v1.31.0
+ * Release Notes", "Compatibility and numerical behavior": caller workspace,
+ * rejected before launch when missing); it holds the work list the device
+ * builds for the call and the persistent CTAs' claim counter.  Its contents
+ * need no initialisation and are rewritten by every call, so calls that
+ * overlap on the GPU need workspaces of their own.
  */
 int attn_fwd_dense(const void *q, const void *k, const void *v, void *o, float *lse,
                    int B, int Sq, int Skv, int Hq, int Hkv, int Dqk, int Dv,
                    const int64_t q_strides[3], const int64_t k_strides[3],
                    const int64_t v_strides[3], const int64_t o_strides[3],
-                   float scale, int causal, void *stream);
+                   float scale, int causal, void *workspace, size_t workspace_bytes,
+                   void *stream);
+
+/* Workspace bytes attn_fwd_dense needs: a 256-byte header plus 16 bytes per
+ * (batch, 128-row query tile, pair of query heads sharing a KV head) work item
+ * (same caller-workspace contract as above).  Host-only arithmetic; 0 for
+ * invalid arguments. */
+size_t attn_fwd_dense_workspace_size(int B, int Sq, int Hq, int Hkv);
 
 /*
  * Ragged / packed THD forward.
@@ -139,7 +154,12 @@ int attn_fwd_ragged(const void *q, const void *k, const void *v, void *o, float 
                     int lse_layout, float scale, int causal,
                     void *workspace, size_t workspace_bytes, void *stream);
 
-/* Workspace bytes attn_fwd_ragged needs for these declared capacities. */
+/* Workspace bytes attn_fwd_ragged needs for these declared capacities: the
+ * caller sizes and owns the scratch, and passes it with the call ("cuDNN
+ * Frontend v1.31.0 Release Notes", "Compatibility and numerical behavior":
+ * direct callers ask for the scratch workspace size, allocate it and pass it;
+ * a missing workspace is rejected before launch).  Host-only arithmetic; 0 for
+ * invalid arguments. */
 size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q,
                                       int Hq, int Hkv);
 
@@ -147,17 +167,20 @@ size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q,
  * attn_fwd_ragged without a workspace argument, for callers that cannot
  * allocate device memory when they call (the release pages have no
  * counterpart; this entry point is specific to this library).  Typical
- * callers: code that runs inside a CUDA stream capture, where a cudaMalloc
- * would invalidate the capture, and plugins or runtimes whose host framework
- * owns all device memory and forbids allocation during execution.
+ * callers: plugins and runtimes whose host framework owns every device
+ * allocation and gives a kernel library none while it executes, and serving
+ * loops that size all their device buffers at start-up and may not call
+ * cudaMalloc afterwards (an allocation there can synchronize the device and
+ * stall the streams already in flight).
  * The work list lives in a 4 MiB array built into the library instead
  * (attn_fwd_ragged_noalloc_max_scratch() returns the size); every GPU that
  * loads the library holds it until the process exits.  Arguments, layouts
  * and results are those of attn_fwd_ragged.
  *  - Capacities whose work list needs more than 4 MiB
  *    (attn_fwd_ragged_workspace_size(...) > 4 MiB) return ATTN_ERR_WORKSPACE.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - The first call on a device that passes the argument checks looks up
+ *    the array's device address (cudaGetSymbolAddress, once per device);
+ *    make that first call before any stream capture.
  *  - All calls share the one array, and each call rewrites it before use.
  *    Calls that overlap on the GPU (e.g. issued on two streams without an
  *    ordering between them) race on it: order them on one stream.
@@ -288,13 +311,20 @@ int attn_fwd_paged_prefill_kv_tables(const void *q, const void *k_pool, const vo
 /* Workspace bytes attn_fwd_paged_prefill needs (the work list of attn_fwd_ragged). */
 size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv);
 
-/* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1). */
+/* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1): the fp32
+ * split partials and the launch order live in caller-owned scratch ("cuDNN
+ * Frontend v1.31.0 Release Notes", "Compatibility and numerical behavior":
+ * split-attention calls require caller workspace, sized by a query). */
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits);
 
 /*
  * A split count for attn_fwd_paged: enough (batch, head, split) blocks to keep
  * num_sms SMs busy through the tail of uneven lengths, while the fp32 partials
- * stay a small fraction of the KV bytes streamed.  Host-only arithmetic.
+ * stay a small fraction of the KV bytes streamed ("cuDNN Frontend v1.31.0
+ * Release Notes", "SDPA: paged KV, split-KV, and engine selection": split
+ * selection from the physical launch capacity and the ragged work, not from a
+ * dense envelope).  Host-only arithmetic; the choice never changes results
+ * beyond rounding.
  */
 int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len,
                               int page_size, int num_sms);

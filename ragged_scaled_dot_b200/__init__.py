@@ -37,7 +37,8 @@ _L3 = ctypes.c_int64 * 3
 SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_fwd_dense": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
-                            _L3, _L3, _L3, _L3, _F, _I, _P]),
+                            _L3, _L3, _L3, _L3, _F, _I, _P, _Z, _P]),
+    "attn_fwd_dense_workspace_size": (_Z, [_I, _I, _I, _I]),
     "attn_fwd_ragged": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _L, _L, _I, _I, _I, _I,
                              _L2, _L2, _L2, _L2, _I, _F, _I, _P, _Z, _P]),
     "attn_fwd_ragged_workspace_size": (_Z, [_I, _I, _L, _I, _I]),
@@ -114,18 +115,25 @@ def _bf16(t, name):
 
 
 # --------------------------------------------------------------------- dense
-def attn_fwd_dense(q, k, v, o, lse=None, *, scale: float, causal: bool, stream=None):
+def attn_fwd_dense_workspace_size(B, Sq, Hq, Hkv) -> int:
+    return int(lib().attn_fwd_dense_workspace_size(B, Sq, Hq, Hkv))
+
+
+def attn_fwd_dense(q, k, v, o, lse=None, *, scale: float, causal: bool, workspace, stream=None):
     """Dense BSHD: q [B,Sq,Hq,Dqk], k [B,Skv,Hkv,Dqk], v [B,Skv,Hkv,Dv],
-    o [B,Sq,Hq,Dv] (strided views allowed), lse fp32 [B,Hq,Sq] contiguous or None."""
+    o [B,Sq,Hq,Dv] (strided views allowed), lse fp32 [B,Hq,Sq] contiguous or None.
+    workspace: uint8 CUDA tensor of attn_fwd_dense_workspace_size(...) bytes."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _bf16(t, n)
     B, Sq, Hq, Dqk = q.shape
     _, Skv, Hkv, _ = k.shape
     Dv = v.shape[-1]
     st = lambda t: _L3(t.stride(0), t.stride(1), t.stride(2))  # noqa: E731
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().attn_fwd_dense(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Sq, Skv, Hq,
                                 Hkv, Dqk, Dv, st(q), st(k), st(v), st(o), float(scale),
-                                int(causal), _stream(stream)), "attn_fwd_dense")
+                                int(causal), _ptr(workspace), ws_bytes, _stream(stream)),
+           "attn_fwd_dense")
 
 
 # -------------------------------------------------------------------- ragged
@@ -161,10 +169,11 @@ def attn_fwd_ragged_noalloc(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_kv, *, max
                             lse_layout: int = ATTN_LSE_PADDED_BSH, total_q=None, total_kv=None,
                             stream=None):
     """attn_fwd_ragged for callers that cannot allocate device memory at call
-    time (inside a stream capture, or under a framework that owns all device
-    memory): the work list goes to a 4 MiB scratch array built into the
-    library.  Calls share that array, so calls that overlap on the GPU race;
-    the first call on a device should come before any stream capture."""
+    time (a host framework that owns every device allocation, or a serving
+    loop that sizes all its buffers at start-up): the work list goes to a
+    4 MiB scratch array built into the library.  Calls share that array, so
+    calls that overlap on the GPU race; the first call on a device should
+    come before any stream capture."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _bf16(t, n)
     B = cu_seqlens_q.numel() - 1

@@ -158,6 +158,47 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     }
 }
 
+// ---------------------------------------------------------------------------
+// Dense BSHD work list, built on the device into the caller's workspace (the
+// same {b, qtile, h0, cost} items and {count, claim counter} header as the
+// ragged list, so the prefill kernel claims dense items the same way).  All
+// sequences have one length, so the order is set by the query tile: groups of
+// kDenseQtGroup query tiles, the group of longest tiles first (longest
+// processing time first: the last items claimed are the cheapest), and inside
+// a group (batch, kv head, query tile longest first, head pair), so the CTAs
+// working at the same time read few (batch, kv head) K/V streams and each
+// stream's prefix is brought from HBM once per group.  Grid-stride over the
+// items; block 0 writes the header.
+// ---------------------------------------------------------------------------
+constexpr int kDenseQtGroup = 8;
+
+__global__ void __launch_bounds__(256) dense_worklist_kernel(int B, int Sq, int Skv, int causal, int Hkv,
+                                                             int pairs_per_group, int heads_per_item, int G,
+                                                             int n_qtiles, int n_items, int* __restrict__ header,
+                                                             int4* __restrict__ items) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        header[0] = n_items;
+        header[1] = 0;
+    }
+    const int per_t = B * Hkv * pairs_per_group;  // items per query tile
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < n_items; idx += gridDim.x * blockDim.x) {
+        const int grp = idx / (kDenseQtGroup * per_t);
+        const int t0 = grp * kDenseQtGroup;
+        const int nt = min(kDenseQtGroup, n_qtiles - t0);  // tiles in this (maybe last) group
+        int rem = idx - t0 * per_t;
+        const int per_bg = nt * pairs_per_group;           // items per (batch, kv head) in the group
+        const int bg = rem / per_bg;
+        rem -= bg * per_bg;
+        const int b = bg / Hkv;
+        const int g = bg - b * Hkv;
+        const int ti = rem / pairs_per_group;
+        const int pr = rem - ti * pairs_per_group;
+        const int t = t0 + ti;
+        const int qt = causal ? (n_qtiles - 1 - t) : t;
+        items[idx] = make_int4(b, qt, g * G + pr * heads_per_item, prefill_n_kv(qt, Sq, Skv, causal));
+    }
+}
+
 // Launch order of a paged decode: sequence indices by cached length, longest
 // first, so the blocks of the longest splits start first and the short ones
 // fill in at the end (list scheduling in longest-processing-time order; the

@@ -239,10 +239,18 @@ const char* attn_status_string(int status) {
 }
 
 // ------------------------------------------------------------------ dense
+size_t attn_fwd_dense_workspace_size(int B, int Sq, int Hq, int Hkv) {
+    if (B <= 0 || Sq < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    // header (item count, claim counter) + one 16-byte item per (batch, query tile, head pair)
+    return (size_t)round_up(256 + (int64_t)B * n_pairs * ((Sq + 127) / 128) * 16, 256);
+}
+
 int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Sq, int Skv,
                    int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[3], const int64_t k_strides[3],
                    const int64_t v_strides[3], const int64_t o_strides[3], float scale, int causal,
-                   void* stream) {
+                   void* workspace, size_t workspace_bytes, void* stream) {
     if (B < 0 || Sq < 0 || Skv < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
     if (!q_strides || !k_strides || !v_strides || !o_strides) return ATTN_ERR_INVALID_ARG;
@@ -254,30 +262,46 @@ int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* 
         if (!stride_ok(q_strides[i]) || !stride_ok(k_strides[i]) || !stride_ok(v_strides[i]) ||
             !stride_ok(o_strides[i]))
             return ATTN_ERR_INVALID_ARG;
+    int hpi, n_pairs;
+    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int n_qtiles = (Sq + 127) / 128;
+    const int64_t n_items = (int64_t)B * n_pairs * n_qtiles;
+    if (n_items >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
+    const size_t need = attn_fwd_dense_workspace_size(B, Sq, Hq, Hkv);
+    if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
     int dev, sms;
     if (int e = setup_device(&dev, &sms)) return e;
     const int D = Dqk;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     PrefillParams pp;
     std::memset(&pp, 0, sizeof(pp));
     if (encode_tok_tiles(&pp.tm_q, q, D, Hq, Sq, B, q_strides[1], q_strides[2], q_strides[0]) ||
         encode_tok_tiles(&pp.tm_k, k, D, Hkv, Skv, B, k_strides[1], k_strides[2], k_strides[0]) ||
         encode_tok_tiles(&pp.tm_v, v, D, Hkv, Skv, B, v_strides[1], v_strides[2], v_strides[0]))
         return ATTN_ERR_INVALID_ARG;
-    int hpi, n_pairs;
-    pair_shape(Hq, Hkv, &hpi, &n_pairs);
+    const int G = Hq / Hkv;
+    char* wsb = static_cast<char*>(workspace);
+    int* header = reinterpret_cast<int*>(wsb);
+    int4* items = reinterpret_cast<int4*>(wsb + 256);
+    {
+        const int64_t want = (n_items + 255) / 256;
+        const int blocks = (int)(want < (int64_t)sms * 4 ? want : (int64_t)sms * 4);
+        b2::dense_worklist_kernel<<<blocks, 256, 0, st>>>(B, Sq, Skv, causal, Hkv, G / hpi, hpi, G, n_qtiles,
+                                                          (int)n_items, header, items);
+        if (int e = launch_status()) return e;
+    }
     pp.mode = 0;
     pp.B = B;
     pp.Hq = Hq;
     pp.Hkv = Hkv;
-    pp.G = Hq / Hkv;
+    pp.G = G;
     pp.heads_per_item = hpi;
-    pp.pairs_per_group = pp.G / hpi;
+    pp.pairs_per_group = G / hpi;
     pp.Sq = Sq;
     pp.Skv = Skv;
-    pp.n_qtiles = (Sq + 127) / 128;
-    const int64_t n_items = (int64_t)B * n_pairs * pp.n_qtiles;
-    if (n_items >= (int64_t)1 << 31) return ATTN_ERR_UNSUPPORTED;
-    pp.n_items = (int)n_items;
+    pp.items = items;
+    pp.header = header;
     pp.o = static_cast<__nv_bfloat16*>(o);
     pp.o_bs = o_strides[0];
     pp.o_ts = o_strides[1];
@@ -287,7 +311,7 @@ int attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* 
     pp.scale_log2 = scale * kLog2e;
     pp.causal = causal;
     const int grid = (int)(n_items < sms ? n_items : sms);
-    return launch_prefill(pp, D, grid, static_cast<cudaStream_t>(stream));
+    return launch_prefill(pp, D, grid, st);
 }
 
 // ----------------------------------------------------------------- ragged
@@ -296,12 +320,18 @@ size_t attn_fwd_ragged_workspace_size(int B, int max_seqlen_q, int64_t total_q, 
     return (size_t)ragged_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv).total;
 }
 
-int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
-                    const int32_t* cu_seqlens_kv, int B, int max_seqlen_q, int max_seqlen_kv, int64_t total_q,
-                    int64_t total_kv, int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[2],
-                    const int64_t k_strides[2], const int64_t v_strides[2], const int64_t o_strides[2],
-                    int lse_layout, float scale, int causal, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+}  // extern "C"
+
+namespace {
+// Host checks of attn_fwd_ragged's arguments, before anything touches the
+// device.  Returns an error status, or ATTN_OK with *empty set when the call
+// has nothing to compute.
+int ragged_check_args(const void* q, const void* k, const void* v, const void* o, const int32_t* cu_seqlens_q,
+                      const int32_t* cu_seqlens_kv, int B, int max_seqlen_q, int max_seqlen_kv, int64_t total_q,
+                      int64_t total_kv, int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[2],
+                      const int64_t k_strides[2], const int64_t v_strides[2], const int64_t o_strides[2],
+                      int lse_layout, float scale, int causal, bool* empty) {
+    *empty = false;
     if (B < 0 || max_seqlen_q < 0 || max_seqlen_kv < 0 || total_q < 0 || total_kv < 0) return ATTN_ERR_INVALID_ARG;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
@@ -311,13 +341,35 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     if (!q_strides || !k_strides || !v_strides || !o_strides) return ATTN_ERR_INVALID_ARG;
     if (Dqk != Dv || (Dqk != 64 && Dqk != 128)) return ATTN_ERR_UNSUPPORTED;
     if (total_q >= ((int64_t)1 << 31) || total_kv >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
-    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) {
+        *empty = true;
+        return ATTN_OK;
+    }
     if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_kv) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
     for (int i = 0; i < 2; ++i)
         if (!stride_ok(q_strides[i]) || !stride_ok(k_strides[i]) || !stride_ok(v_strides[i]) ||
             !stride_ok(o_strides[i]))
             return ATTN_ERR_INVALID_ARG;
+    return ATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* cu_seqlens_q,
+                    const int32_t* cu_seqlens_kv, int B, int max_seqlen_q, int max_seqlen_kv, int64_t total_q,
+                    int64_t total_kv, int Hq, int Hkv, int Dqk, int Dv, const int64_t q_strides[2],
+                    const int64_t k_strides[2], const int64_t v_strides[2], const int64_t o_strides[2],
+                    int lse_layout, float scale, int causal, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    bool empty = false;
+    if (int e = ragged_check_args(q, k, v, o, cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv, total_q,
+                                  total_kv, Hq, Hkv, Dqk, Dv, q_strides, k_strides, v_strides, o_strides, lse_layout,
+                                  scale, causal, &empty))
+        return e;
+    if (empty) return ATTN_OK;
+    const int lse_base = lse_layout & ~ATTN_LSE_LOG2;
     const size_t need = attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
     if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
@@ -389,6 +441,15 @@ int attn_fwd_ragged_noalloc(const void* q, const void* k, const void* v, void* o
                             int Dv, const int64_t q_strides[2], const int64_t k_strides[2],
                             const int64_t v_strides[2], const int64_t o_strides[2], int lse_layout, float scale,
                             int causal, void* stream) {
+    // every host check and the empty-problem return come before the first
+    // device call (the scratch address lookup), so an invalid or empty call
+    // never does that lookup
+    bool empty = false;
+    if (int e = ragged_check_args(q, k, v, o, cu_seqlens_q, cu_seqlens_kv, B, max_seqlen_q, max_seqlen_kv, total_q,
+                                  total_kv, Hq, Hkv, Dqk, Dv, q_strides, k_strides, v_strides, o_strides, lse_layout,
+                                  scale, causal, &empty))
+        return e;
+    if (empty) return ATTN_OK;
     const size_t need = attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
     if (need > kNoAllocScratchBytes) return ATTN_ERR_WORKSPACE;  // work list would not fit 4 MiB
     void* scratch = nullptr;

@@ -1,13 +1,15 @@
 // prefill.cuh -- forward attention prefill on tcgen05 tensor cores (sm_100a).
 //
-// One persistent CTA per SM claims work items one at a time.  A work item is
+// One persistent CTA per SM claims work items one at a time from a list built
+// on the device (a claim counter in the caller's workspace).  A work item is
 // (sequence b, query tile of 128 rows, up to two query heads of one GQA group):
 // the two heads share every K/V tile, so each K/V byte brought on chip feeds
 // two 128x128 score tiles ("cuDNN Frontend v1.30.0 Release Notes", "New:
-// decode tiles", GQA packing; the grouping here is our own).  Items are
-// ordered (sequence longest first, kv head, query tile longest first, head
-// pair), so the CTAs working at the same time share one sequence-head's K/V
-// in L2 and the long items start first.
+// decode tiles", GQA packing; the grouping here is our own).  Ragged and paged
+// items are ordered (sequence longest first, kv head, query tile longest
+// first, head pair), dense items (group of query tiles longest first, batch,
+// kv head, query tile, head pair), so the CTAs working at the same time share
+// few sequence-heads' K/V in L2 and the long items start first.
 //
 // Warp roles (320 threads):
 //   warp 0      claims items, publishes them to the other roles through a
@@ -59,12 +61,10 @@ struct PrefillParams {
     int heads_per_item;   // 2 when G is even, else 1
     int pairs_per_group;  // G / heads_per_item
     int Sq, Skv;          // dense
-    int n_qtiles;         // dense: ceil(Sq / 128)
-    int n_items;          // dense: number of work items
     const int32_t* cu_q;
     const int32_t* cu_kv;
-    const int4* items;  // ragged: work list {b, qtile, h0, cost}
-    int* header;        // ragged: [0] item count, [1] claim counter
+    const int4* items;  // work list {b, qtile, h0, cost}, built on the device
+    int* header;        // [0] item count, [1] claim counter
     __nv_bfloat16* o;
     int64_t o_bs, o_ts, o_hs;  // element strides (batch, token, head)
     float* lse;
@@ -108,37 +108,18 @@ __device__ __forceinline__ int prefill_n_kv(int qt, int Lq, int Lkv, int causal)
 }
 
 __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx, PrefillItem& it) {
+    const int4 w = p.items[idx];
+    it.b = w.x;
+    it.qt = w.y;
+    it.h0 = w.z;
     if (p.mode == 0) {
-        // dense: groups of kQtGroup query tiles, the longest group first; inside a group
-        // (batch, kv head, query tile longest first, head pair).  The static round-robin
-        // assignment then hands out items of nearly equal length side by side, and the
-        // CTAs working at the same time share few (batch, kv head) K/V streams in L2.
-        constexpr int kQtGroup = 4;
-        const int per_t = p.B * p.Hkv * p.pairs_per_group;  // items per query tile
-        const int grp = idx / (kQtGroup * per_t);
-        const int t0 = grp * kQtGroup;
-        const int nt = min(kQtGroup, p.n_qtiles - t0);       // tiles in this (maybe last) group
-        int rem = idx - t0 * per_t;
-        const int per_bg = nt * p.pairs_per_group;           // items per (batch, kv head) in the group
-        const int bg = rem / per_bg;
-        rem -= bg * per_bg;
-        it.b = bg / p.Hkv;
-        const int g = bg - it.b * p.Hkv;
-        const int ti = rem / p.pairs_per_group;
-        const int pr = rem - ti * p.pairs_per_group;
-        const int t = t0 + ti;
-        it.qt = p.causal ? (p.n_qtiles - 1 - t) : t;
-        it.h0 = g * p.G + pr * p.heads_per_item;
+        // dense: sequence b is batch b of the 5D maps, every sequence Sq x Skv
         it.q_tok0 = it.qt * 128;
         it.kv_tok0 = 0;
         it.batch = it.b;
         it.Lq = p.Sq;
         it.Lkv = p.Skv;
     } else {
-        const int4 w = p.items[idx];
-        it.b = w.x;
-        it.qt = w.y;
-        it.h0 = w.z;
         const int q0 = __ldg(p.cu_q + it.b), q1 = __ldg(p.cu_q + it.b + 1);
         it.Lq = q1 - q0;
         it.q_tok0 = q0 + it.qt * 128;
@@ -280,13 +261,13 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
 
     if (warp == 0 && lane == 0) {
         // ---------------------------------------------- scheduler + producer
-        const int n_items = (p.mode == 0) ? p.n_items : p.header[0];
+        const int n_items = p.header[0];
         int kv_it = 0, q_it = 0;
         bool ok = true;
         for (int k = 0; ok; ++k) {
             const int r = k % NRING;
             if (!mbar_wait(b_iempty0 + 8 * r, ((k / NRING) & 1) ^ 1, abort_flag)) break;
-            int idx = (p.mode == 0) ? (int)blockIdx.x + k * (int)gridDim.x : atomicAdd(p.header + 1, 1);
+            int idx = atomicAdd(p.header + 1, 1);
             if (idx >= n_items) idx = -1;
             item_ring[r] = idx;
             mbar_arrive(b_ifull0 + 8 * r);

@@ -141,7 +141,9 @@ def dense_gpu(q, k, v, scale, causal, o=None, lse=None):
         o = torch.full((B, Sq, Hq, v.shape[-1]), float("nan"), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.full((B, Hq, Sq), float("nan"), dtype=torch.float32, device=q.device)
-    rsd.attn_fwd_dense(q, k, v, o, lse, scale=scale, causal=causal)
+    ws = torch.empty(rsd.attn_fwd_dense_workspace_size(B, Sq, Hq, k.shape[2]), dtype=torch.uint8, device=q.device)
+    ws.fill_(0xFF)  # the call must build its list and reset its counter itself
+    rsd.attn_fwd_dense(q, k, v, o, lse, scale=scale, causal=causal, workspace=ws)
     torch.cuda.synchronize()
     return o, lse
 

@@ -72,16 +72,33 @@ L3 = ctypes.c_int64 * 3
 def test_dense_rejects_bad_args_on_host(lib):
     st = L3(8 * 4 * 64, 4 * 64, 64)
     f = lib.attn_fwd_dense
+    fake = ctypes.c_void_p(0x100000)   # never dereferenced: rejected before launch
+    ws = ctypes.c_void_p(0x100100)     # 256-byte aligned
     # Hq not a multiple of Hkv
-    assert f(None, None, None, None, None, 1, 8, 8, 3, 2, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, 1, 8, 8, 3, 2, 64, 64, st, st, st, st, 1.0, 1, None, 0, None) == rsd.ATTN_ERR_INVALID_ARG
     # unsupported head dim
-    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 96, 96, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_UNSUPPORTED
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 96, 96, st, st, st, st, 1.0, 1, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED
     # non-finite scale
-    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, float("nan"), 1, None) == rsd.ATTN_ERR_INVALID_ARG
-    # empty problem is a no-op
-    assert f(None, None, None, None, None, 0, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_OK
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, float("nan"), 1, None, 0, None) == rsd.ATTN_ERR_INVALID_ARG
+    # empty problem is a no-op, workspace or not
+    assert f(None, None, None, None, None, 0, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None, 0, None) == rsd.ATTN_OK
     # null pointers with a real shape
-    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None) == rsd.ATTN_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None, 0, None) == rsd.ATTN_ERR_INVALID_ARG
+    # the work list needs a workspace: missing, too small or misaligned is refused before launch
+    need = rsd.attn_fwd_dense_workspace_size(1, 8, 4, 1)
+    assert f(fake, fake, fake, fake, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, None, 0, None) == rsd.ATTN_ERR_WORKSPACE
+    assert f(fake, fake, fake, fake, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1, ws, need - 1, None) == rsd.ATTN_ERR_WORKSPACE
+    assert f(fake, fake, fake, fake, None, 1, 8, 8, 4, 1, 64, 64, st, st, st, st, 1.0, 1,
+             ctypes.c_void_p(0x100010), need, None) == rsd.ATTN_ERR_WORKSPACE
+
+
+def test_dense_workspace_size(lib):
+    # header + one 16-byte item per (batch, 128-row query tile, head pair)
+    n = rsd.attn_fwd_dense_workspace_size(8, 4096, 32, 8)
+    assert n == 256 + 8 * 32 * 16 * 16 and n % 256 == 0
+    assert rsd.attn_fwd_dense_workspace_size(2, 100, 3, 1) == 256 + 256   # G odd: one head per item, 2*1*3 items
+    assert rsd.attn_fwd_dense_workspace_size(0, 100, 4, 1) == 0
+    assert rsd.attn_fwd_dense_workspace_size(1, 100, 3, 2) == 0             # Hq % Hkv != 0
 
 
 def test_ragged_requires_workspace(lib):

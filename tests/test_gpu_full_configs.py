@@ -19,7 +19,9 @@ def test_dense_prefill_full_size():
     q, k, v = synth.make_dense(w, DEV)
     o = torch.full_like(q, float("nan"))
     lse = torch.full((w.B, w.Hq, w.S), float("nan"), dtype=torch.float32, device=DEV)
-    rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True)
+    ws = torch.full((rsd.attn_fwd_dense_workspace_size(w.B, w.S, w.Hq, w.Hkv),), 0xFF, dtype=torch.uint8,
+                    device=DEV)
+    rsd.attn_fwd_dense(q, k, v, o, lse, scale=w.scale, causal=True, workspace=ws)
     torch.cuda.synchronize()
     assert not torch.isnan(o).any() and not torch.isnan(lse).any()
     rng = np.random.default_rng(0)
