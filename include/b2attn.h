@@ -371,6 +371,25 @@ int attn_selftest_bounded_wait(uint64_t timeout_ns, void *stream);
  */
 int attn_selftest_exp2(const float *t, float *y, int64_t n, void *stream);
 
+/*
+ * Diagnostic of the page-table address generation: for n sampled logical keys
+ * (b_idx[i], t_idx[i]) writes out[3i], out[3i+1], out[3i+2] = (physical page,
+ * row in the page, 8-row group of the pool) computed by the same device
+ * functions the paged producers use, so a test can check them against the
+ * definition bit for bit ("cuDNN Frontend v1.31.0 Release Notes", "SDPA:
+ * paged KV, split-KV, and engine selection": key t of sequence b is row
+ * t % page_size of page page_table[b * page_table_stride + t / page_size]; the
+ * group is page * groups_per_page + row / 8).  A table entry outside
+ * [0, num_pages) gives page = group = -1 and records ATTN_ERR_DEVICE_INPUT,
+ * as it does in the producers.  Every (b_idx[i], t_idx[i]) must address an
+ * entry of the table (t_idx >= 0).  All arrays are DEVICE memory; out holds
+ * 3n int64.  num_pages * groups_per_page must stay below 2^31
+ * (ATTN_ERR_UNSUPPORTED otherwise).
+ */
+int attn_selftest_page_coords(const int32_t *page_table, int64_t page_table_stride, int page_size,
+                              int64_t num_pages, int groups_per_page, const int32_t *b_idx,
+                              const int32_t *t_idx, int64_t n, int64_t *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

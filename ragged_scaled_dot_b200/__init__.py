@@ -60,6 +60,7 @@ SIGNATURES = {
     "attn_get_device_error": (_I, [_P]),
     "attn_selftest_bounded_wait": (_I, [_U64, _P]),
     "attn_selftest_exp2": (_I, [_P, _P, _L, _P]),
+    "attn_selftest_page_coords": (_I, [_P, _L, _I, _L, _I, _P, _P, _L, _P, _P]),
 }
 
 _lib = None
@@ -331,3 +332,14 @@ def attn_selftest_exp2(t, y, stream=None):
     """y = 2**t through the prefill softmax's FMA-pipe exponential (fp32 CUDA tensors)."""
     _check(lib().attn_selftest_exp2(_ptr(t), _ptr(y), int(t.numel()), _stream(stream)),
            "attn_selftest_exp2")
+
+
+def attn_selftest_page_coords(page_table, b_idx, t_idx, out, *, page_size: int, num_pages: int,
+                              groups_per_page: int, stream=None):
+    """(page, row, 8-row group) of sampled logical keys, as the paged producers
+    compute them: page_table int32 CUDA [B, max_pages], b_idx / t_idx int32 CUDA [n],
+    out int64 CUDA [n, 3]."""
+    _check(lib().attn_selftest_page_coords(_ptr(page_table), int(page_table.stride(0)), int(page_size),
+                                           int(num_pages), int(groups_per_page), _ptr(b_idx), _ptr(t_idx),
+                                           int(b_idx.numel()), _ptr(out), _stream(stream)),
+           "attn_selftest_page_coords")

@@ -16,6 +16,7 @@
 #include "aux_kernels.cuh"
 #include "decode.cuh"
 #include "decode_mla.cuh"
+#include "paging.cuh"
 
 namespace {
 
@@ -826,6 +827,21 @@ int attn_selftest_exp2(const float* t, float* y, int64_t n, void* stream) {
     const int64_t blocks = (n / 2 + 255) / 256 + 1;
     if (blocks > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     b2::selftest_exp2_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(t, y, n);
+    return launch_status();
+}
+
+int attn_selftest_page_coords(const int32_t* page_table, int64_t page_table_stride, int page_size,
+                              int64_t num_pages, int groups_per_page, const int32_t* b_idx, const int32_t* t_idx,
+                              int64_t n, int64_t* out, void* stream) {
+    if (n < 0 || page_size <= 0 || num_pages <= 0 || groups_per_page <= 0 || page_table_stride < 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (num_pages * groups_per_page >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (n == 0) return ATTN_OK;
+    if (!page_table || !b_idx || !t_idx || !out) return ATTN_ERR_INVALID_ARG;
+    const int64_t want = (n + 255) / 256;
+    const unsigned blocks = (unsigned)(want < 1024 ? want : 1024);
+    b2::page_coords_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        page_table, page_table_stride, page_size, num_pages, groups_per_page, b_idx, t_idx, n, out);
     return launch_status();
 }
 

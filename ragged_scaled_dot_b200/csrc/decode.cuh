@@ -18,6 +18,7 @@
 // longest splits start first and the short ones fill the tail.
 #pragma once
 
+#include "paging.cuh"
 #include "ptx.cuh"
 
 namespace b2 {
@@ -81,12 +82,9 @@ __device__ __forceinline__ void decode_issue_chunk(const DecodeParams& p, const 
     const int nkeys = min(64, hi - t0);
     for (int r = 0; r < nkeys; r += p.box_rows) {
         const int t = t0 + r;
-        int page = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
-        if (page < 0 || (int64_t)page >= p.num_pages) {
-            record_status(ATTN_ERR_DEVICE_INPUT);
-            page = -1;  // out of range: TMA fills the box with zeros
-        }
-        const int slot = t % p.page_size;
+        // out of range: page -1, and TMA fills the box with zeros
+        const int page = page_checked(page_lookup(table, table_stride, b, t, p.page_size), p.num_pages);
+        const int slot = page_slot(t, p.page_size);
         for (int cb = 0; cb < ncol_blocks; ++cb)
             tma_load_4d(dst + cb * block_bytes + (uint32_t)r * 128u, map, bar, cb * 64, slot, g, page);
     }

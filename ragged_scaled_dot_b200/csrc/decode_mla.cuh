@@ -101,7 +101,7 @@ __device__ __forceinline__ uint32_t mla_fetch_pages(const DecodeParams& p, const
         const int t = t0 + i * p.box_rows;
         pg[i] = -1;
         if (i < np && t < hi) {
-            pg[i] = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
+            pg[i] = page_lookup(table, table_stride, b, t, p.page_size);
             live |= 1u << i;
         }
     }
@@ -119,13 +119,8 @@ __device__ __forceinline__ void mla_issue(const DecodeParams& p, const CUtensorM
         if (i < np) {
             int page = -1, tok = 0;
             if ((live >> i) & 1u) {
-                page = pg[i];
-                if (page < 0 || (int64_t)page >= p.num_pages) {
-                    record_status(ATTN_ERR_DEVICE_INPUT);
-                    page = -1;
-                } else {
-                    tok = (t0 + i * p.box_rows) % p.page_size;
-                }
+                page = page_checked(pg[i], p.num_pages);
+                if (page >= 0) tok = page_slot(t0 + i * p.box_rows, p.page_size);
             }
             tma_load_5d(dst + (uint32_t)(i * nblk * p.box_rows) * 128u, map, bar, 0, tok, blk0, 0, page);
         }

@@ -47,6 +47,7 @@
 // past the causal diagonal are never loaded.
 #pragma once
 
+#include "paging.cuh"
 #include "ptx.cuh"
 
 namespace b2 {
@@ -150,11 +151,8 @@ __device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const C
         const int t = t0 + i * p.box_rows;
         int gg = p.n_groups;
         if (t < Lkv) {
-            const int page = __ldg(table + (int64_t)b * table_stride + t / p.page_size);
-            if (page < 0 || (int64_t)page >= p.num_pages)
-                record_status(ATTN_ERR_DEVICE_INPUT);
-            else
-                gg = page * p.groups_per_page + (t % p.page_size) / 8;
+            const int page = page_checked(page_lookup(table, table_stride, b, t, p.page_size), p.num_pages);
+            if (page >= 0) gg = page_group(page, page_slot(t, p.page_size), p.groups_per_page);
         }
         tma_load_5d(dst + (uint32_t)i * box_bytes, map, bar, 0, 0, 0, gg, g);
     }

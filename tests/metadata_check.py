@@ -1,0 +1,146 @@
+"""Host-side checks of the metadata the library builds on the device: the
+prefill work lists (ragged, paged-prefill and dense), the split-decode launch
+order and the page-table coordinates.  Each expected value is computed here
+from the rule the header and the design state, with plain Python, not with the
+library.  Used by ``test_gpu_metadata.py`` (device lists) and
+``test_metadata_check_cpu.py`` (the checks themselves reject planted mistakes).
+
+Work-list rules (one item = (sequence b, 128-row query tile qt, first query
+head h0 of the pair, KV tiles the item visits)):
+  * a query tile visits every 128-key tile that holds a key some row of the
+    tile may see (bottom-right causal: row i of Lq sees keys j <= i + Lkv - Lq);
+  * ragged / paged: a sequence's items form one contiguous run ordered
+    (kv head, query tile longest first, head pair); runs are ordered by the
+    sequence's total tile steps (capped at 4095), most first, ties in any order;
+  * dense: groups of 8 query tiles, the group of longest tiles first, inside a
+    group (batch, kv head, query tile longest first, head pair);
+  * header[0] = item count; after the prefill ran, header[1] = item count +
+    number of persistent CTAs (each CTA makes one claim past the end).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+SORT_CAP = 4095
+DENSE_GROUP = 8
+
+
+def heads_per_item(Hq, Hkv):
+    return 2 if (Hq // Hkv) % 2 == 0 else 1
+
+
+def kv_tiles_visited(qt, Lq, Lkv, causal):
+    """128-key tiles holding at least one key visible to a row of query tile qt."""
+    if Lkv <= 0:
+        return 0
+    if not causal:
+        return (Lkv + 127) // 128
+    last_row = min(Lq, (qt + 1) * 128) - 1
+    max_key = min(Lkv - 1, last_row + Lkv - Lq)
+    return 0 if max_key < 0 else max_key // 128 + 1
+
+
+def sequence_block(b, Lq, Lkv, Hq, Hkv, causal):
+    """The run of items of sequence b, in its documented order."""
+    G = Hq // Hkv
+    hpi = heads_per_item(Hq, Hkv)
+    nqt = (Lq + 127) // 128
+    out = []
+    for g in range(Hkv):
+        for t in range(nqt):
+            qt = nqt - 1 - t
+            for pr in range(G // hpi):
+                out.append((b, qt, g * G + pr * hpi, kv_tiles_visited(qt, Lq, Lkv, causal)))
+    return out
+
+
+def sequence_key(Lq, Lkv, causal):
+    nqt = (Lq + 127) // 128
+    return min(SORT_CAP, sum(kv_tiles_visited(qt, Lq, Lkv, causal) for qt in range(nqt)))
+
+
+def check_sequence_list(items, count, lq, lkv, Hq, Hkv, causal):
+    """items: int array [n, 4] as the device wrote them; count: header[0].
+    Raises AssertionError on any deviation: a dropped, duplicated or altered
+    item, a run out of its internal order, or runs out of key order."""
+    items = np.asarray(items, dtype=np.int64).reshape(-1, 4)
+    blocks = {b: sequence_block(b, int(lq[b]), int(lkv[b]), Hq, Hkv, causal) for b in range(len(lq))}
+    want = sum(len(v) for v in blocks.values())
+    assert count == want, f"item count {count}, expected {want}"
+    assert len(items) >= count
+    seen = set()
+    pos = 0
+    prev_key = None
+    while pos < count:
+        b = int(items[pos, 0])
+        assert 0 <= b < len(lq), f"item {pos}: sequence {b} out of range"
+        assert b not in seen, f"sequence {b} appears in two runs"
+        blk = blocks[b]
+        assert len(blk) > 0, f"sequence {b} has no queries but has items"
+        got = [tuple(int(x) for x in r) for r in items[pos:pos + len(blk)]]
+        assert got == blk, f"run of sequence {b} at {pos} differs from its expected items"
+        key = sequence_key(int(lq[b]), int(lkv[b]), causal)
+        assert prev_key is None or key <= prev_key, f"sequence {b} (key {key}) after key {prev_key}"
+        prev_key = key
+        seen.add(b)
+        pos += len(blk)
+    missing = [b for b, v in blocks.items() if v and b not in seen]
+    assert not missing, f"sequences without their run: {missing}"
+
+
+def dense_list(B, Sq, Skv, Hq, Hkv, causal):
+    """The dense list in its documented order."""
+    G = Hq // Hkv
+    hpi = heads_per_item(Hq, Hkv)
+    nqt = (Sq + 127) // 128
+    out = []
+    for t0 in range(0, nqt, DENSE_GROUP):
+        ts = range(t0, min(nqt, t0 + DENSE_GROUP))
+        for b in range(B):
+            for g in range(Hkv):
+                for t in ts:
+                    qt = nqt - 1 - t if causal else t
+                    for pr in range(G // hpi):
+                        out.append((b, qt, g * G + pr * hpi, kv_tiles_visited(qt, Sq, Skv, causal)))
+    return out
+
+
+def check_dense_list(items, count, B, Sq, Skv, Hq, Hkv, causal):
+    want = dense_list(B, Sq, Skv, Hq, Hkv, causal)
+    assert count == len(want), f"item count {count}, expected {len(want)}"
+    got = [tuple(int(x) for x in r) for r in np.asarray(items, dtype=np.int64).reshape(-1, 4)[:count]]
+    assert got == want, "dense list differs from its expected order"
+
+
+def ragged_max_tiles(B, max_sq, total_q):
+    """Query tiles the declared capacities allow (the launch is sized by them)."""
+    return min(total_q // 128 + B, B * ((max_sq + 127) // 128))
+
+
+def decode_order_shift(max_kv_len):
+    shift = 0
+    while (max_kv_len >> shift) >= 4096:
+        shift += 1
+    return shift
+
+
+def check_decode_order(order, kv_lens, max_kv_len):
+    """A permutation of the sequences, longest first by bucket min(4095, L >> shift)."""
+    order = [int(x) for x in order]
+    assert sorted(order) == list(range(len(kv_lens))), "launch order is not a permutation"
+    shift = decode_order_shift(max_kv_len)
+    keys = [min(4095, max(0, min(int(kv_lens[b]), max_kv_len)) >> shift) for b in order]
+    assert all(a >= b for a, b in zip(keys, keys[1:])), "launch order is not longest first"
+
+
+def page_coords(table, b_idx, t_idx, page_size, num_pages, groups_per_page):
+    """(page or -1, row, 8-row group or -1) of logical keys (b, t) by the page-table rule."""
+    out = []
+    for b, t in zip(b_idx, t_idx):
+        page = int(table[int(b), int(t) // page_size])
+        row = int(t) % page_size
+        if page < 0 or page >= num_pages:
+            out.append((-1, row, -1))
+        else:
+            out.append((page, row, page * groups_per_page + row // 8))
+    return np.array(out, dtype=np.int64).reshape(-1, 3)
