@@ -282,7 +282,7 @@ def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
     smax = int(lq.max())
     o = torch.empty_like(q)
     lse = torch.empty((w.B, smax, w.Hq), dtype=torch.float32, device=dev)
-    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv), dtype=torch.uint8,
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv, w.Dqk, 1), dtype=torch.uint8,
                      device=dev)
     cud = torch.as_tensor(cu_q, device=dev)
     pt = torch.as_tensor(table, device=dev)
@@ -298,6 +298,47 @@ def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
     info = {"workload": w.notes, "flop_per_step": flops, "query_tokens": int(T),
             "kv_tokens": int(L.sum()), "total_pages": int(kp.shape[0]), "traffic_basis_gb": io_gb}
     return Part("paged_prefill", "TFLOP/s", flops / 1e12, 3, step, None, info), None
+
+
+def make_mixed(torch, rsd, synth, dev, seed_offset, num_sms, subset="all"):
+    """The mixed decode / chunked-prefill batch over a paged cache through
+    attn_fwd_paged_prefill: subset "all" (one call for every row), "short"
+    (only the 1-4-query rows: K/V GB/s of the split-KV decode kernel) or
+    "chunks" (only the 1024-query chunks: TFLOP/s of the prefill kernel)."""
+    w0 = synth.WORKLOADS["mixed_batch"]
+    w = synth.Workload(**{**w0.__dict__, "seed": w0.seed + seed_offset})
+    q, kp, vp, table, kl, cu_q, lq = synth.make_mixed_batch(w, dev, subset)
+    L = kl.astype(np.int64)
+    T = int(cu_q[-1])
+    smax = int(lq.max())
+    o = torch.empty_like(q)
+    lse = torch.empty((T, w.Hq), dtype=torch.float32, device=dev)
+    maxL = int(L.max())
+    n_short = int(np.sum((lq >= 1) & (lq <= 4)))
+    S = rsd.attn_paged_suggest_splits(max(1, n_short), w.Hq, w.Hkv, w.Dqk, w.Dv, maxL, w.page_size, num_sms)
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv, w.Dqk, S),
+                     dtype=torch.uint8, device=dev)
+    cud = torch.as_tensor(cu_q, device=dev)
+    pt = torch.as_tensor(table, device=dev)
+    kld = torch.as_tensor(kl, device=dev)
+
+    def step():
+        rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, cud, pt, kld, max_seqlen_q=smax, page_size=w.page_size,
+                                   max_kv_len=maxL, scale=w.scale, causal=True, workspace=ws, num_splits=S,
+                                   lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    flops = prefill_flops(lq, L, w.Hq, w.Dqk)
+    short = (lq >= 1) & (lq <= 4)
+    kv_short = float(np.sum(L[short])) * w.Hkv * (w.Dqk + w.Dv) * 2
+    qmax = min(4, 64 // (w.Hq // w.Hkv), smax)
+    launches = 1 + (1 + (2 if S > 1 else 0) if qmax > 0 else 0) + (1 if smax > qmax else 0)
+    info = {"workload": w.notes, "subset": subset, "num_splits_short_rows": S, "query_tokens": T,
+            "short_sequences": n_short, "chunk_sequences": int(np.sum(lq > 4)), "flop_per_step": flops,
+            "kv_bytes_short_rows": kv_short, "traffic_basis_gb": kv_short / 1e9}
+    if subset == "short":
+        info["bytes_per_unit"] = f"{w.Hkv * (w.Dqk + w.Dv) * 2} B of K/V per cached token of a short sequence"
+        return Part("mixed_short_rows", "GB/s", kv_short / 1e9, launches, step, None, info)
+    name = "mixed_chunks" if subset == "chunks" else "mixed_batch"
+    return Part(name, "TFLOP/s", flops / 1e12, launches, step, None, info)
 
 
 def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
@@ -562,6 +603,8 @@ def run_ours(args):
         extras.append(make_paged_prefill(torch, rsd, synth, dev, off)[0])
         mla, _ = make_paged(torch, rsd, synth, dev, off, "mla_decode", num_sms)
         extras.append(mla)
+        for subset in ("all", "short", "chunks"):
+            extras.append(make_mixed(torch, rsd, synth, dev, off, num_sms, subset))
     torch.cuda.synchronize()
 
     results = {}
@@ -689,6 +732,9 @@ def run_one(args):
         part = make_dense_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
     elif args.only == "paged_prefill":
         part = make_paged_prefill(torch, rsd, synth, "cuda", 0, args.batch)[0]
+    elif args.only.startswith("mixed"):
+        part = make_mixed(torch, rsd, synth, "cuda", 0, num_sms,
+                          {"mixed_batch": "all", "mixed_short_rows": "short", "mixed_chunks": "chunks"}[args.only])
     else:
         part = make_paged(torch, rsd, synth, "cuda", 0, args.only, num_sms, args.batch)[0]
     total_ms, per = time_part(torch, part, args.steps, args.warmup, None, 1)
@@ -748,7 +794,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "paged_prefill",
-                                       "mla_decode"],
+                                       "mla_decode", "mixed_batch", "mixed_short_rows", "mixed_chunks"],
                     help="profiling: time one part only and print its own line")
     ap.add_argument("--batch", type=int, default=0, help="profiling: override the part's batch size")
     args = ap.parse_args()

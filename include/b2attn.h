@@ -262,10 +262,11 @@ int attn_fwd_paged_kv_tables(const void *q, const void *k_pool, const void *v_po
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Ragged queries over a paged K/V cache: chunked prefill and multi-token
- * decode ("cuDNN Frontend v1.31.0 Release Notes", "SDPA: paged KV, split-KV,
- * and engine selection": paged K/V for prefill; "cuDNN Frontend v1.28.0
- * release notes", ragged / THD queries).  Sequence b has
+ * Ragged queries over a paged K/V cache: chunked prefill, decode and
+ * multi-token decode rows in one batch ("cuDNN Frontend v1.31.0 Release
+ * Notes", "SDPA: paged KV, split-KV, and engine selection": paged K/V for
+ * prefill, prepared paged D128 THD split-KV; "cuDNN Frontend v1.28.0 release
+ * notes", ragged / THD queries).  Sequence b has
  * Lq_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] queries, the LAST Lq_b positions
  * of its kv_lens[b] cached keys: with causal, query i sees keys
  * j <= i + kv_lens[b] - Lq_b (bottom-right); Lq_b > kv_lens[b] leaves the
@@ -273,6 +274,15 @@ int attn_fwd_paged_kv_tables(const void *q, const void *k_pool, const void *v_po
  *   q, o: packed THD [total_q, Hq, D], (token, head) element strides.
  *   k_pool / v_pool, page_table, kv_lens: as for attn_fwd_paged (DEVICE).
  *   lse / lse_layout: as for attn_fwd_ragged.
+ * Short rows: the sequences with 1 <= Lq_b <= qmax queries, qmax =
+ * min(4, 64 / (Hq / Hkv), max_seqlen_q) (none when Hq / Hkv > 64), run on the
+ * split-KV decode kernel, which streams their keys once per KV head with the
+ * G query heads x Lq_b tokens as the rows of its tiles; the others run on the
+ * tensor-core prefill kernel in 128-row query tiles.  The split is decided on
+ * the device from cu_seqlens_q (no host read); results do not depend on it.
+ * num_splits (>= 1) splits the keys of each short sequence as attn_fwd_paged
+ * does (fp32 partials in the workspace, merged by LSE); it does not affect
+ * the other sequences.  attn_paged_suggest_splits gives a count.
  * Supported: D = Dqk = Dv in {64, 128}, Hq % Hkv == 0, page_size dividing 128
  * (at least 8) or a multiple of 128, and pools whose page stride is a whole
  * number of 8-row groups (page stride % (8 * row stride) == 0, the same for K
@@ -288,7 +298,7 @@ int attn_fwd_paged_prefill(const void *q, const void *k_pool, const void *v_pool
                            int page_size, int64_t num_pages, int max_kv_len,
                            const int64_t q_strides[2], const int64_t o_strides[2],
                            const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
-                           int lse_layout, float scale, int causal,
+                           int lse_layout, float scale, int causal, int num_splits,
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
@@ -306,10 +316,17 @@ int attn_fwd_paged_prefill_kv_tables(const void *q, const void *k_pool, const vo
                                      int max_kv_len, const int64_t q_strides[2],
                                      const int64_t o_strides[2], const int64_t k_pool_strides[3],
                                      const int64_t v_pool_strides[3], int lse_layout, float scale,
-                                     int causal, void *workspace, size_t workspace_bytes, void *stream);
+                                     int causal, int num_splits, void *workspace, size_t workspace_bytes,
+                                     void *stream);
 
-/* Workspace bytes attn_fwd_paged_prefill needs (the work list of attn_fwd_ragged). */
-size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv);
+/* Workspace bytes attn_fwd_paged_prefill needs: the prefill work list (as for
+ * attn_fwd_ragged) and, with num_splits > 1, the fp32 partials of the short
+ * rows (B * qmax * Hq rows of D floats per split) and their launch order
+ * (caller workspace as in "cuDNN Frontend v1.31.0 Release Notes",
+ * "Compatibility and numerical behavior").  Host-only arithmetic; 0 for
+ * invalid arguments. */
+size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv,
+                                             int D, int num_splits);
 
 /* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1): the fp32
  * split partials and the launch order live in caller-owned scratch ("cuDNN

@@ -51,10 +51,10 @@ SIGNATURES = {
                                       _L2, _L2, _L3, _L3, _F, _I, _P, _Z, _P]),
     "attn_fwd_paged_workspace_size": (_Z, [_I, _I, _I, _I]),
     "attn_fwd_paged_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _L, _I, _I, _I, _I, _L, _I,
-                                    _L2, _L2, _L3, _L3, _I, _F, _I, _P, _Z, _P]),
+                                    _L2, _L2, _L3, _L3, _I, _F, _I, _I, _P, _Z, _P]),
     "attn_fwd_paged_prefill_kv_tables": (_I, [_P, _P, _P, _P, _P, _P, _P, _L, _P, _L, _P, _I, _I, _L, _I, _I,
-                                              _I, _I, _L, _I, _L2, _L2, _L3, _L3, _I, _F, _I, _P, _Z, _P]),
-    "attn_fwd_paged_prefill_workspace_size": (_Z, [_I, _I, _L, _I, _I]),
+                                              _I, _I, _L, _I, _L2, _L2, _L3, _L3, _I, _F, _I, _I, _P, _Z, _P]),
+    "attn_fwd_paged_prefill_workspace_size": (_Z, [_I, _I, _L, _I, _I, _I, _I]),
     "attn_paged_suggest_splits": (_I, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "attn_split_merge": (_I, [_P, _P, _I, _L, _I, _P, _L, _P, _P]),
     "attn_get_device_error": (_I, [_P]),
@@ -255,19 +255,21 @@ def attn_fwd_paged_kv_tables(q, k_pool, v_pool, o, lse, k_page_table, v_page_tab
         float(scale), int(num_splits), _ptr(workspace), ws_bytes, _stream(stream)), "attn_fwd_paged_kv_tables")
 
 
-def attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv) -> int:
-    return int(lib().attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv))
+def attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv, D=128, num_splits=1) -> int:
+    return int(lib().attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv, D, num_splits))
 
 
 def attn_fwd_paged_prefill(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, kv_lens, *,
                            max_seqlen_q: int, page_size: int, max_kv_len: int, scale: float,
-                           causal: bool, workspace, lse_layout: int = ATTN_LSE_PADDED_BSH,
-                           kv_layout: str = "HND", total_q=None, stream=None):
-    """Ragged queries over a paged cache (chunked prefill, multi-token decode):
-    q [T,Hq,D] packed by cu_seqlens_q (int32 CUDA [B+1]); sequence b's queries are
-    the last Lq_b positions of its kv_lens[b] keys (bottom-right causal).  Pools 4D
-    in kv_layout, page_table int32 CUDA [B,max_pages], o [T,Hq,D], lse as in
-    attn_fwd_ragged.  workspace: uint8 CUDA tensor."""
+                           causal: bool, workspace, num_splits: int = 1,
+                           lse_layout: int = ATTN_LSE_PADDED_BSH, kv_layout: str = "HND", total_q=None,
+                           stream=None):
+    """Ragged queries over a paged cache (chunked prefill, decode and multi-token
+    decode rows): q [T,Hq,D] packed by cu_seqlens_q (int32 CUDA [B+1]); sequence b's
+    queries are the last Lq_b positions of its kv_lens[b] keys (bottom-right causal).
+    Pools 4D in kv_layout, page_table int32 CUDA [B,max_pages], o [T,Hq,D], lse as in
+    attn_fwd_ragged.  Sequences of at most 4 queries run split-KV with num_splits
+    splits.  workspace: uint8 CUDA tensor of attn_fwd_paged_prefill_workspace_size(...)."""
     for t, n in ((q, "q"), (k_pool, "k_pool"), (v_pool, "v_pool"), (o, "o")):
         _bf16(t, n)
     B = cu_seqlens_q.numel() - 1
@@ -281,13 +283,13 @@ def attn_fwd_paged_prefill(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, 
         int(page_table.stride(0)), _ptr(kv_lens), B, int(max_seqlen_q), int(total_q), Hq, Hkv, D,
         int(page_size), int(num_pages), int(max_kv_len), _L2(q.stride(0), q.stride(1)),
         _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout), pool_strides(v_pool, kv_layout),
-        int(lse_layout), float(scale), int(causal), _ptr(workspace), ws_bytes, _stream(stream)),
-        "attn_fwd_paged_prefill")
+        int(lse_layout), float(scale), int(causal), int(num_splits), _ptr(workspace), ws_bytes,
+        _stream(stream)), "attn_fwd_paged_prefill")
 
 
 def attn_fwd_paged_prefill_kv_tables(q, k_pool, v_pool, o, lse, cu_seqlens_q, k_page_table, v_page_table,
                                      kv_lens, *, max_seqlen_q: int, page_size: int, max_kv_len: int,
-                                     scale: float, causal: bool, workspace,
+                                     scale: float, causal: bool, workspace, num_splits: int = 1,
                                      lse_layout: int = ATTN_LSE_PADDED_BSH, kv_layout: str = "HND",
                                      total_q=None, stream=None):
     """attn_fwd_paged_prefill with independent K and V page tables."""
@@ -304,8 +306,8 @@ def attn_fwd_paged_prefill_kv_tables(q, k_pool, v_pool, o, lse, cu_seqlens_q, k_
         int(k_page_table.stride(0)), _ptr(v_page_table), int(v_page_table.stride(0)), _ptr(kv_lens), B,
         int(max_seqlen_q), int(total_q), Hq, Hkv, D, int(page_size), int(num_pages), int(max_kv_len),
         _L2(q.stride(0), q.stride(1)), _L2(o.stride(0), o.stride(1)), pool_strides(k_pool, kv_layout),
-        pool_strides(v_pool, kv_layout), int(lse_layout), float(scale), int(causal), _ptr(workspace), ws_bytes,
-        _stream(stream)), "attn_fwd_paged_prefill_kv_tables")
+        pool_strides(v_pool, kv_layout), int(lse_layout), float(scale), int(causal), int(num_splits),
+        _ptr(workspace), ws_bytes, _stream(stream)), "attn_fwd_paged_prefill_kv_tables")
 
 
 # --------------------------------------------------------------------- merge

@@ -2,6 +2,7 @@
 // LSE fill, the split-KV LSE merge and the bounded-wait self-test.
 #pragma once
 
+#include "prefill.cuh"
 #include "ptx.cuh"
 
 namespace b2 {
@@ -47,12 +48,17 @@ __device__ __forceinline__ int seq_cost_key(int lq, int lk, int causal) {
     return min(cost, kSortBuckets - 1);
 }
 
+// Query tiles a sequence of lq queries gives the prefill kernel: none for the
+// sequences of 1..short_q queries that the split-KV decode kernel takes
+// (short_q = 0: the prefill kernel takes every sequence).
+__device__ __forceinline__ int prefill_qtiles(int lq, int short_q) { return lq <= short_q ? 0 : (lq + 127) >> 7; }
+
 __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv,
     const int32_t* __restrict__ kv_lens, int B, int max_sq,
     int max_skv, int64_t total_q, int64_t total_kv, int causal, int Hkv, int pairs_per_group,
     int heads_per_item, int G, int* __restrict__ header, int4* __restrict__ items,
-    int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles) {
+    int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles, int short_q) {
     __shared__ int hist[kSortBuckets];
     __shared__ int warp_sums[32];
     __shared__ int n_tiles_sh;
@@ -68,8 +74,8 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         int nqt = 0, key = 0;
         if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) {
             const int lq = cu_q[b + 1] - cu_q[b];
-            nqt = (lq + 127) >> 7;
-            key = seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal);
+            nqt = prefill_qtiles(lq, short_q);
+            key = nqt ? seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal) : 0;
         } else {
             record_status(ATTN_ERR_DEVICE_INPUT);
         }
@@ -91,8 +97,8 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         int nqt = 0, key = 0;
         if (ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) {
             const int lq = cu_q[b + 1] - cu_q[b];
-            nqt = (lq + 127) >> 7;
-            key = seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal);
+            nqt = prefill_qtiles(lq, short_q);
+            key = nqt ? seq_cost_key(lq, seq_kv_len(cu_kv, kv_lens, b), causal) : 0;
         }
         const int r = atomicAdd(&hist[key], 1);
         rank_of[b] = r;
@@ -142,7 +148,8 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     for (int b = tid; b < B; b += blockDim.x) {
         if (!ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) continue;
         const int lq = cu_q[b + 1] - cu_q[b], lk = seq_kv_len(cu_kv, kv_lens, b);
-        const int nqt = (lq + 127) >> 7;
+        const int nqt = prefill_qtiles(lq, short_q);
+        if (nqt == 0) continue;
         const int tile0 = sorted_nqt[rank_of[b]];  // first tile slot of this sequence
         if (tile0 + nqt > max_tiles) continue;
         const int64_t base = (int64_t)tile0 * n_pairs;
@@ -208,13 +215,19 @@ __global__ void __launch_bounds__(256) dense_worklist_kernel(int B, int Sq, int 
 // which block runs a (sequence, split), never what it computes.  One block of
 // 1024 threads.
 __global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restrict__ kv_lens, int B, int max_kv_len,
-                                                         int shift, int32_t* __restrict__ order) {
+                                                         int shift, int32_t* __restrict__ order,
+                                                         const int32_t* __restrict__ cu_q, int qmax) {
     __shared__ int hist[kSortBuckets];
     __shared__ int warp_sums[32];
     const int tid = threadIdx.x;
-    // bucket 0 holds the longest sequences
+    // bucket 0 holds the longest sequences; with ragged queries (cu_q), the
+    // sequences the decode kernel skips (not 1..qmax queries) count as empty
     auto bucket = [&](int b) {
-        const int L = max(0, min(__ldg(kv_lens + b), max_kv_len));
+        int L = max(0, min(__ldg(kv_lens + b), max_kv_len));
+        if (cu_q != nullptr) {
+            const int lq = __ldg(cu_q + b + 1) - __ldg(cu_q + b);
+            if (lq < 1 || lq > qmax) L = 0;
+        }
         return kSortBuckets - 1 - min(kSortBuckets - 1, L >> shift);
     };
     for (int i = tid; i < kSortBuckets; i += blockDim.x) hist[i] = 0;
@@ -281,24 +294,24 @@ __global__ void lse_padded_fill_kernel(const int32_t* __restrict__ cu_q, int B, 
 // Computed in the log2 domain: exp(x) = 2^(x log2 e).
 // ---------------------------------------------------------------------------
 template <int DV>
-__global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ o_part,
-                                                          const float* __restrict__ lse_part,
-                                                          int S, int64_t R,
-                                                          __nv_bfloat16* __restrict__ o,
-                                                          int64_t o_row_stride,
-                                                          float* __restrict__ lse) {
-    constexpr float LOG2E = 1.4426950408889634f;
-    constexpr int VEC = (DV % 128 == 0) ? 4 : 2;  // floats per vector access
-    constexpr int NV = DV / (32 * VEC);           // vector accesses per lane
+struct MergeVec {
+    static constexpr int VEC = (DV % 128 == 0) ? 4 : 2;  // floats per vector access
+    static constexpr int NV = DV / (32 * VEC);           // vector accesses per lane
     static_assert(NV >= 1 && DV % (32 * VEC) == 0, "unsupported Dv");
-    const int64_t r = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (r >= R) return;
+};
+
+// The merge of row r by one warp: lane holds columns VEC * (lane + 32 i) + e in
+// acc[i][e]; returns the natural-log LSE of the row (-inf when every partial is).
+template <int DV>
+__device__ __forceinline__ float merge_row(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                                           int S, int64_t R, int64_t r, int lane,
+                                           float (&acc)[MergeVec<DV>::NV][MergeVec<DV>::VEC]) {
+    constexpr float LOG2E = 1.4426950408889634f;
+    constexpr int VEC = MergeVec<DV>::VEC, NV = MergeVec<DV>::NV;
     float M = -INFINITY;
     for (int s = lane; s < S; s += 32) M = fmaxf(M, lse_part[(int64_t)s * R + r]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float acc[NV][VEC];
 #pragma unroll
     for (int i = 0; i < NV; ++i)
 #pragma unroll
@@ -329,7 +342,14 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
             }
         }
     }
-    __nv_bfloat16* dst = o + r * o_row_stride;
+    return L;
+}
+
+// One merged row as bf16 at dst (8-byte aligned), the lane's columns as in merge_row.
+template <int DV>
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, int lane,
+                                               const float (&acc)[MergeVec<DV>::NV][MergeVec<DV>::VEC]) {
+    constexpr int VEC = MergeVec<DV>::VEC, NV = MergeVec<DV>::NV;
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
         const int e0 = VEC * (lane + 32 * i);
@@ -342,6 +362,21 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
             *reinterpret_cast<uint32_t*>(dst + e0) = pack_bf16(acc[i][0], acc[i][1]);
         }
     }
+}
+
+template <int DV>
+__global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ o_part,
+                                                          const float* __restrict__ lse_part,
+                                                          int S, int64_t R,
+                                                          __nv_bfloat16* __restrict__ o,
+                                                          int64_t o_row_stride,
+                                                          float* __restrict__ lse) {
+    const int64_t r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= R) return;
+    float acc[MergeVec<DV>::NV][MergeVec<DV>::VEC];
+    const float L = merge_row<DV>(o_part, lse_part, S, R, r, lane, acc);
+    store_row_bf16<DV>(o + r * o_row_stride, lane, acc);
     if (lse != nullptr && lane == 0) lse[r] = L;
 }
 

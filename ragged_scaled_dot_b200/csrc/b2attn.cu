@@ -69,12 +69,12 @@ int setup_device(int* dev_out, int* sms_out) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(b2::prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::PrefillCfg<128>::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(b2::decode_gqa_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     b2::DecodeCfg<64>::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(b2::decode_gqa_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     b2::DecodeCfg<128>::SMEM);
+        const void* decode_kernels[6] = {(const void*)b2::decode_gqa_kernel<64, 1>, (const void*)b2::decode_gqa_kernel<64, 2>,
+                                         (const void*)b2::decode_gqa_kernel<64, 4>, (const void*)b2::decode_gqa_kernel<128, 1>,
+                                         (const void*)b2::decode_gqa_kernel<128, 2>, (const void*)b2::decode_gqa_kernel<128, 4>};
+        for (int i = 0; i < 6 && e == cudaSuccess; ++i)
+            e = cudaFuncSetAttribute(decode_kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     i < 3 ? b2::DecodeCfg<64>::SMEM : b2::DecodeCfg<128>::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(b2::decode_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::MlaTcCfg::SMEM);
@@ -201,6 +201,49 @@ int noalloc_scratch(void** out) {
     }
     *out = g_noalloc_ptr[dev];
     return ATTN_OK;
+}
+
+// Launches the GQA decode kernel with RT 16-row m-tiles (1, 2 or 4) over grid
+// (num_splits, Hkv, B).
+int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, cudaStream_t st) {
+    if (D == 128) {
+        if (RT == 1) b2::decode_gqa_kernel<128, 1><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+        else if (RT == 2) b2::decode_gqa_kernel<128, 2><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<128, 4><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+    } else {
+        if (RT == 1) b2::decode_gqa_kernel<64, 1><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+        else if (RT == 2) b2::decode_gqa_kernel<64, 2><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<64, 4><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+    }
+    return launch_status();
+}
+
+// GQA decode maps over a pool: (d, slot, head, page), 64-column boxes of one
+// page's min(page_size, 64) rows.
+int encode_decode_pool_maps(DecodeParams& dp, const void* k_pool, const void* v_pool, int Dqk, int Dv, int page_size,
+                            int Hkv, int64_t num_pages, const int64_t k_pool_strides[3],
+                            const int64_t v_pool_strides[3]) {
+    const int box_rows = page_size < 64 ? page_size : 64;
+    const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
+    const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
+    const int64_t sk[3] = {k_pool_strides[1], k_pool_strides[2], k_pool_strides[0]};
+    if (encode_4d(&dp.tm_k, k_pool, dk, sk, box)) return ATTN_ERR_INVALID_ARG;
+    const uint64_t dv[4] = {(uint64_t)Dv, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
+    const int64_t sv[3] = {v_pool_strides[1], v_pool_strides[2], v_pool_strides[0]};
+    if (encode_4d(&dp.tm_v, v_pool, dv, sv, box)) return ATTN_ERR_INVALID_ARG;
+    dp.box_rows = box_rows;
+    return ATTN_OK;
+}
+
+// Ragged queries over a paged cache: the sequences of 1..qmax queries go to
+// the split-KV decode kernel (G query heads x qmax tokens as the MMA rows, at
+// most 64), the others to the prefill kernel.  0 when G > 64 (no routing).
+int routed_qmax(int G, int max_seqlen_q) {
+    if (G > 64) return 0;
+    int q = 64 / G;
+    if (q > 4) q = 4;
+    if (q > max_seqlen_q) q = max_seqlen_q;
+    return q;
 }
 
 // Launches the prefill kernel for an already-filled PrefillParams.
@@ -400,7 +443,7 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
         cu_seqlens_q, cu_seqlens_kv, nullptr, B, max_seqlen_q, max_seqlen_kv, total_q, total_kv, causal, Hkv, G / hpi,
         hpi, G, header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
-        max_tiles);
+        max_tiles, 0);
     if (int e = launch_status()) return e;
     if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
         const int64_t n = (int64_t)B * max_seqlen_q * Hq;
@@ -463,8 +506,40 @@ int attn_fwd_ragged_noalloc(const void* q, const void* k, const void* v, void* o
 size_t attn_fwd_ragged_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
 
 // ------------------------------------------------ paged prefill (chunked)
-size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv) {
-    return attn_fwd_ragged_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
+}  // extern "C"
+
+namespace {
+// Paged-prefill workspace: the ragged work list, then (routed short rows with
+// splits) partial O fp32 [S][B*qmax*Hq][D], partial LSE [S][B*qmax*Hq] and the
+// decode launch order [B], each 256-byte aligned.
+struct PagedPrefillWs {
+    RaggedWs rw;
+    int qmax;
+    int64_t part_off, lse_off, order_off, total;
+};
+PagedPrefillWs paged_prefill_ws_layout(int B, int max_sq, int64_t total_q, int Hq, int Hkv, int D, int num_splits) {
+    PagedPrefillWs w;
+    w.rw = ragged_ws_layout(B, max_sq, total_q, Hq, Hkv);
+    w.qmax = routed_qmax(Hq / Hkv, max_sq);
+    w.part_off = w.lse_off = w.order_off = w.total = w.rw.total;
+    if (w.qmax > 0 && num_splits > 1) {
+        const int64_t R = (int64_t)B * w.qmax * Hq;
+        w.lse_off = w.part_off + round_up(R * num_splits * D * 4, 256);
+        w.order_off = w.lse_off + round_up(R * num_splits * 4, 256);
+        w.total = w.order_off + round_up((int64_t)B * 4, 256);
+    }
+    return w;
+}
+}  // namespace
+
+extern "C" {
+
+size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv, int D,
+                                             int num_splits) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_seqlen_q < 0 || total_q < 0 || D <= 0 ||
+        num_splits < 1)
+        return 0;
+    return (size_t)paged_prefill_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv, D, num_splits).total;
 }
 
 int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
@@ -472,13 +547,13 @@ int attn_fwd_paged_prefill(const void* q, const void* k_pool, const void* v_pool
                            const int32_t* kv_lens, int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv,
                            int D, int page_size, int64_t num_pages, int max_kv_len, const int64_t q_strides[2],
                            const int64_t o_strides[2], const int64_t k_pool_strides[3],
-                           const int64_t v_pool_strides[3], int lse_layout, float scale, int causal,
+                           const int64_t v_pool_strides[3], int lse_layout, float scale, int causal, int num_splits,
                            void* workspace, size_t workspace_bytes, void* stream) {
     return attn_fwd_paged_prefill_kv_tables(q, k_pool, v_pool, o, lse, cu_seqlens_q, page_table, page_table_stride,
                                             page_table, page_table_stride, kv_lens, B, max_seqlen_q, total_q, Hq,
                                             Hkv, D, page_size, num_pages, max_kv_len, q_strides, o_strides,
-                                            k_pool_strides, v_pool_strides, lse_layout, scale, causal, workspace,
-                                            workspace_bytes, stream);
+                                            k_pool_strides, v_pool_strides, lse_layout, scale, causal, num_splits,
+                                            workspace, workspace_bytes, stream);
 }
 
 int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const void* v_pool, void* o, float* lse,
@@ -488,11 +563,12 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
                                      int64_t total_q, int Hq, int Hkv, int D, int page_size, int64_t num_pages,
                                      int max_kv_len, const int64_t q_strides[2], const int64_t o_strides[2],
                                      const int64_t k_pool_strides[3], const int64_t v_pool_strides[3],
-                                     int lse_layout, float scale, int causal, void* workspace,
+                                     int lse_layout, float scale, int causal, int num_splits, void* workspace,
                                      size_t workspace_bytes, void* stream) {
     if (B < 0 || max_seqlen_q < 0 || total_q < 0 || max_kv_len < 0 || num_pages < 0) return ATTN_ERR_INVALID_ARG;
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+    if (num_splits < 1 || num_splits > 4096) return ATTN_ERR_INVALID_ARG;
     const int lse_base = lse_layout & ~ATTN_LSE_LOG2;
     if (lse_base != ATTN_LSE_PADDED_BSH && lse_base != ATTN_LSE_PACKED_TH && lse_base != ATTN_LSE_PACKED_HT)
         return ATTN_ERR_INVALID_ARG;
@@ -502,6 +578,7 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     // a page box of min(page_size, 128) rows: whole 8-row groups that tile a 128-key tile
     if (!(page_size % 128 == 0 || (128 % page_size == 0 && page_size >= 8))) return ATTN_ERR_UNSUPPORTED;
     if (total_q >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
     if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
     if (!q || !k_pool || !v_pool || !o || !cu_seqlens_q || !k_page_table || !v_page_table || !kv_lens)
         return ATTN_ERR_INVALID_ARG;
@@ -521,14 +598,91 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         gk != gv || gk < page_size / 8)
         return ATTN_ERR_UNSUPPORTED;
     if ((int64_t)num_pages * gk >= ((int64_t)1 << 31)) return ATTN_ERR_UNSUPPORTED;
-    const size_t need = attn_fwd_paged_prefill_workspace_size(B, max_seqlen_q, total_q, Hq, Hkv);
-    if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+    const PagedPrefillWs wl = paged_prefill_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv, D, num_splits);
+    if (workspace == nullptr || workspace_bytes < (size_t)wl.total) return ATTN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
     int dev, sms;
     if (int e = setup_device(&dev, &sms)) return e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int R = page_size < 128 ? page_size : 128;
+    const int G = Hq / Hkv;
+    const int qmax = wl.qmax;
+    char* wsb = static_cast<char*>(workspace);
 
+    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
+        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
+        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
+        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
+        if (int e = launch_status()) return e;
+    }
+    const int dev_lse_layout = (lse_base == ATTN_LSE_PADDED_BSH) ? 1 : (lse_base == ATTN_LSE_PACKED_TH) ? 2 : 3;
+
+    // ---- sequences of 1..qmax queries (decode, multi-token decode): split-KV decode kernel
+    if (qmax > 0) {
+        DecodeParams dp;
+        std::memset(&dp, 0, sizeof(dp));
+        if (int e = encode_decode_pool_maps(dp, k_pool, v_pool, D, D, page_size, Hkv, num_pages, k_pool_strides,
+                                            v_pool_strides))
+            return e;
+        dp.q = static_cast<const __nv_bfloat16*>(q);
+        dp.q_bs = q_strides[0];
+        dp.q_hs = q_strides[1];
+        dp.page_table = k_page_table;
+        dp.pt_stride = k_page_table_stride;
+        dp.v_page_table = v_page_table;
+        dp.v_pt_stride = v_page_table_stride;
+        dp.kv_lens = kv_lens;
+        dp.cu_q = cu_seqlens_q;
+        dp.total_q = total_q;
+        dp.qmax = qmax;
+        dp.causal = causal;
+        dp.B = B;
+        dp.Hq = Hq;
+        dp.Hkv = Hkv;
+        dp.G = G;
+        dp.page_size = page_size;
+        dp.num_pages = num_pages;
+        dp.max_kv_len = max_kv_len;
+        dp.num_splits = num_splits;
+        dp.scale_log2 = scale * kLog2e;
+        dp.o = static_cast<__nv_bfloat16*>(o);
+        dp.o_bs = o_strides[0];
+        dp.o_hs = o_strides[1];
+        dp.lse = lse;
+        dp.lse_layout = dev_lse_layout;
+        dp.lse_smax = max_seqlen_q;
+        dp.lse_hs = total_q;
+        dp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
+        if (num_splits > 1) {
+            dp.o_part = reinterpret_cast<float*>(wsb + wl.part_off);
+            dp.lse_part = reinterpret_cast<float*>(wsb + wl.lse_off);
+            int32_t* order = reinterpret_cast<int32_t*>(wsb + wl.order_off);
+            int shift = 0;
+            while ((max_kv_len >> shift) >= 4096) ++shift;
+            b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order, cu_seqlens_q, qmax);
+            if (int e = launch_status()) return e;
+            dp.order = order;
+        }
+        int RT = (G * qmax + 15) / 16;
+        if (RT == 3) RT = 4;
+        if (int e = launch_decode_gqa(dp, D, RT, dim3(num_splits, Hkv, B), st)) return e;
+        if (num_splits > 1) {
+            const int64_t rows = (int64_t)B * qmax * Hq;
+            const unsigned blocks = (unsigned)((rows + 7) / 8);
+            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+            if (D == 128)
+                b2::split_merge_thd_kernel<128><<<blocks, 256, 0, st>>>(
+                    dp.o_part, dp.lse_part, num_splits, cu_seqlens_q, B, qmax, Hq, total_q, ob, o_strides[0],
+                    o_strides[1], lse, dev_lse_layout, max_seqlen_q, total_q, dp.lse_log2);
+            else
+                b2::split_merge_thd_kernel<64><<<blocks, 256, 0, st>>>(
+                    dp.o_part, dp.lse_part, num_splits, cu_seqlens_q, B, qmax, Hq, total_q, ob, o_strides[0],
+                    o_strides[1], lse, dev_lse_layout, max_seqlen_q, total_q, dp.lse_log2);
+            if (int e = launch_status()) return e;
+        }
+    }
+
+    // ---- the other sequences: tcgen05 prefill kernel over page boxes
     PrefillParams pp;
     std::memset(&pp, 0, sizeof(pp));
     if (encode_tok_tiles(&pp.tm_q, q, D, Hq, total_q, 1, q_strides[0], q_strides[1],
@@ -545,23 +699,17 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     }
     int hpi, n_pairs;
     pair_shape(Hq, Hkv, &hpi, &n_pairs);
-    const int G = Hq / Hkv;
     const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
-    const RaggedWs wl = ragged_ws_layout(B, max_seqlen_q, total_q, Hq, Hkv);
-    char* wsb = static_cast<char*>(workspace);
     int* header = reinterpret_cast<int*>(wsb);
-    int4* items = reinterpret_cast<int4*>(wsb + wl.items_off);
+    int4* items = reinterpret_cast<int4*>(wsb + wl.rw.items_off);
     b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
         cu_seqlens_q, nullptr, kv_lens, B, max_seqlen_q, max_kv_len, total_q, 0, causal, Hkv, G / hpi, hpi, G,
-        header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
-        max_tiles);
+        header, items, reinterpret_cast<int*>(wsb + wl.rw.sorted_off), reinterpret_cast<int*>(wsb + wl.rw.rank_off),
+        max_tiles, qmax);
     if (int e = launch_status()) return e;
-    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
-        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
-        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
-        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
-        if (int e = launch_status()) return e;
-    }
+    // the work-list kernel also validates every sequence; with all of them short
+    // (max_seqlen_q <= qmax) its list is empty and the prefill kernel has nothing to do
+    if (qmax > 0 && max_seqlen_q <= qmax) return ATTN_OK;
     pp.mode = 2;
     pp.B = B;
     pp.Hq = Hq;
@@ -712,13 +860,9 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
         const uint32_t bv[5] = {64, (uint32_t)box_rows, (uint32_t)b2::MlaTcCfg::VB, 1, 1};
         if (encode_5d(&dp.tm_v, v_pool, dv, sv, bv)) return ATTN_ERR_INVALID_ARG;
     } else {
-        const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
-        const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
-        const int64_t sk[3] = {k_pool_strides[1], k_pool_strides[2], k_pool_strides[0]};
-        if (encode_4d(&dp.tm_k, k_pool, dk, sk, box)) return ATTN_ERR_INVALID_ARG;
-        const uint64_t dv[4] = {(uint64_t)Dv, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
-        const int64_t sv[3] = {v_pool_strides[1], v_pool_strides[2], v_pool_strides[0]};
-        if (encode_4d(&dp.tm_v, v_pool, dv, sv, box)) return ATTN_ERR_INVALID_ARG;
+        if (int e = encode_decode_pool_maps(dp, k_pool, v_pool, Dqk, Dv, page_size, Hkv, num_pages, k_pool_strides,
+                                            v_pool_strides))
+            return e;
     }
     dp.q = static_cast<const __nv_bfloat16*>(q);
     dp.q_bs = q_strides[0];
@@ -728,6 +872,7 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     dp.v_page_table = v_page_table;
     dp.v_pt_stride = v_page_table_stride;
     dp.kv_lens = kv_lens;
+    dp.qmax = 1;  // one query token per sequence (cu_q stays null)
     dp.B = B;
     dp.Hq = Hq;
     dp.Hkv = Hkv;
@@ -752,7 +897,7 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
                                                     round_up(R * num_splits * 4, 256));
         int shift = 0;
         while ((max_kv_len >> shift) >= 4096) ++shift;
-        b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order);
+        b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order, nullptr, 1);
         if (int e = launch_status()) return e;
         dp.order = order;
     }
@@ -775,11 +920,8 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, b2::decode_mla_tc_kernel, dp) != cudaSuccess) return ATTN_ERR_LAUNCH;
     } else {
-        dim3 grid(num_splits, Hkv, B);
-        if (Dqk == 128)
-            b2::decode_gqa_kernel<128><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
-        else
-            b2::decode_gqa_kernel<64><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+        // the G <= 16 query heads of a KV head fill one m16 tile
+        if (int e = launch_decode_gqa(dp, Dqk, 1, dim3(num_splits, Hkv, B), st)) return e;
     }
     if (int e = launch_status()) return e;
     if (num_splits > 1)

@@ -119,6 +119,12 @@ WORKLOADS = {
         lengths=(1024,), len_range=(8192, 65536), page_size=64, causal=True,
         notes="chunked prefill: 16 sequences, a 1024-token chunk at the end of a paged cache of "
               "U[8192, 65536] keys, page 64, H=32/8 D=128, bottom-right causal"),
+    "mixed_batch": Workload(
+        "mixed_batch", "paged", seed=7, B=64, Hq=32, Hkv=8, Dqk=128, Dv=128,
+        lengths=(1024, 1, 2, 4), len_range=(4096, 32768), page_size=64, causal=True,
+        notes="mixed decode / chunked-prefill batch over a paged cache: 64 sequences with cached "
+              "lengths U[4096, 32768]; sequences 0-15 a 1024-query chunk, the other 48 decode rows "
+              "of 1, 2, 4 queries in turn; page 64, H=32/8 D=128, bottom-right causal"),
     "mla_decode": Workload(
         "mla_decode", "paged", seed=5, B=64, Hq=128, Hkv=1, Dqk=576, Dv=512,
         len_range=(4096, 65536), page_size=64, causal=False, v_aliases_k=True,
@@ -177,3 +183,34 @@ def make_paged(w: Workload, device="cpu", kv_lens=None, extra_pages: int = 0):
     else:
         v_pool = normal_bf16((P, w.Hkv, w.page_size, w.Dv), w.seed * 10 + 3, device)
     return q, k_pool, v_pool, table, L.astype(np.int32)
+
+
+def mixed_query_lengths(w: Workload, kv_lens, subset: str = "all"):
+    """Query lengths of the mixed batch: sequences 0..B/4-1 take a chunk of
+    w.lengths[0] queries, the others the short lengths w.lengths[1:] in turn
+    (capped by each cached length).  subset: "all", "short" (chunks set to 0)
+    or "chunks" (short rows set to 0)."""
+    kv_lens = np.asarray(kv_lens, dtype=np.int64)
+    n_chunk = w.B // 4
+    short = list(w.lengths[1:])
+    lq = np.array([w.lengths[0] if b < n_chunk else short[(b - n_chunk) % len(short)] for b in range(w.B)],
+                  dtype=np.int64)
+    if subset == "short":
+        lq[:n_chunk] = 0
+    elif subset == "chunks":
+        lq[n_chunk:] = 0
+    return np.minimum(lq, kv_lens)
+
+
+def make_mixed_batch(w: Workload, device="cpu", subset: str = "all"):
+    """Mixed-batch inputs: q [sum Lq, Hq, D] packed, HND pools, page table and
+    kv_lens (host), cu_q and the query lengths (host).  Sequences a subset
+    leaves out keep their cache but have no queries."""
+    L = uniform_lengths(w.B, w.len_range[0], w.len_range[1], w.seed)
+    lq = mixed_query_lengths(w, L, subset)
+    cu_q = cu_seqlens(lq)
+    table, total = page_table(L, w.page_size, w.seed)
+    q = normal_bf16((max(1, int(cu_q[-1])), w.Hq, w.Dqk), w.seed * 10 + 1, device)
+    k_pool = normal_bf16((total, w.Hkv, w.page_size, w.Dqk), w.seed * 10 + 2, device)
+    v_pool = normal_bf16((total, w.Hkv, w.page_size, w.Dv), w.seed * 10 + 3, device)
+    return q, k_pool, v_pool, table, L.astype(np.int32), cu_q, lq

@@ -9,7 +9,9 @@ Work-list rules (one item = (sequence b, 128-row query tile qt, first query
 head h0 of the pair, KV tiles the item visits)):
   * a query tile visits every 128-key tile that holds a key some row of the
     tile may see (bottom-right causal: row i of Lq sees keys j <= i + Lkv - Lq);
-  * ragged / paged: a sequence's items form one contiguous run ordered
+  * ragged / paged: sequences of 1..short_q queries have no items (ragged
+    queries over a paged cache send them to the split-KV decode kernel,
+    short_q = min(4, 64 / G, max_seqlen_q)); a sequence's items form one contiguous run ordered
     (kv head, query tile longest first, head pair); runs are ordered by the
     sequence's total tile steps (capped at 4095), most first, ties in any order;
   * dense: groups of 8 query tiles, the group of longest tiles first, inside a
@@ -26,6 +28,7 @@ DENSE_GROUP = 8
 
 
 def heads_per_item(Hq, Hkv):
+    """Query heads per work item: the two heads of a pair that share a KV head (one when G is odd)."""
     return 2 if (Hq // Hkv) % 2 == 0 else 1
 
 
@@ -40,11 +43,16 @@ def kv_tiles_visited(qt, Lq, Lkv, causal):
     return 0 if max_key < 0 else max_key // 128 + 1
 
 
-def sequence_block(b, Lq, Lkv, Hq, Hkv, causal):
+def routed_qmax(G, max_seqlen_q):
+    """Query count up to which ragged queries over a paged cache take the decode kernel."""
+    return 0 if G > 64 else min(4, 64 // G, max_seqlen_q)
+
+
+def sequence_block(b, Lq, Lkv, Hq, Hkv, causal, short_q=0):
     """The run of items of sequence b, in its documented order."""
     G = Hq // Hkv
     hpi = heads_per_item(Hq, Hkv)
-    nqt = (Lq + 127) // 128
+    nqt = 0 if Lq <= short_q else (Lq + 127) // 128
     out = []
     for g in range(Hkv):
         for t in range(nqt):
@@ -54,17 +62,17 @@ def sequence_block(b, Lq, Lkv, Hq, Hkv, causal):
     return out
 
 
-def sequence_key(Lq, Lkv, causal):
-    nqt = (Lq + 127) // 128
+def sequence_key(Lq, Lkv, causal, short_q=0):
+    nqt = 0 if Lq <= short_q else (Lq + 127) // 128
     return min(SORT_CAP, sum(kv_tiles_visited(qt, Lq, Lkv, causal) for qt in range(nqt)))
 
 
-def check_sequence_list(items, count, lq, lkv, Hq, Hkv, causal):
+def check_sequence_list(items, count, lq, lkv, Hq, Hkv, causal, short_q=0):
     """items: int array [n, 4] as the device wrote them; count: header[0].
     Raises AssertionError on any deviation: a dropped, duplicated or altered
     item, a run out of its internal order, or runs out of key order."""
     items = np.asarray(items, dtype=np.int64).reshape(-1, 4)
-    blocks = {b: sequence_block(b, int(lq[b]), int(lkv[b]), Hq, Hkv, causal) for b in range(len(lq))}
+    blocks = {b: sequence_block(b, int(lq[b]), int(lkv[b]), Hq, Hkv, causal, short_q) for b in range(len(lq))}
     want = sum(len(v) for v in blocks.values())
     assert count == want, f"item count {count}, expected {want}"
     assert len(items) >= count
@@ -79,7 +87,7 @@ def check_sequence_list(items, count, lq, lkv, Hq, Hkv, causal):
         assert len(blk) > 0, f"sequence {b} has no queries but has items"
         got = [tuple(int(x) for x in r) for r in items[pos:pos + len(blk)]]
         assert got == blk, f"run of sequence {b} at {pos} differs from its expected items"
-        key = sequence_key(int(lq[b]), int(lkv[b]), causal)
+        key = sequence_key(int(lq[b]), int(lkv[b]), causal, short_q)
         assert prev_key is None or key <= prev_key, f"sequence {b} (key {key}) after key {prev_key}"
         prev_key = key
         seen.add(b)

@@ -145,7 +145,7 @@ def test_kv_table_entry_points_validate_both_tables(lib):
 
     def pre(vt, vstride):
         return g(fake, fake, fake, fake, None, fake, fake, 64, vt, vstride, fake, 2, 512, 600, 32, 4, 128, 64,
-                 100, 4096, q3, q3, kp3, kp3, rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, None, 0, None)
+                 100, 4096, q3, q3, kp3, kp3, rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, 1, None, 0, None)
 
     assert pre(fake, 64) == rsd.ATTN_ERR_WORKSPACE
     assert pre(None, 64) == rsd.ATTN_ERR_INVALID_ARG
@@ -200,13 +200,13 @@ def test_paged_prefill_rejects_bad_args_on_host(lib):
     fake = ctypes.c_void_p(0x100000)
     q2 = L2(32 * 128, 128)
     kp = L3(4 * 64 * 128, 128, 64 * 128)          # HND [pages, 4 heads, 64 rows, 128]
-    args = dict(B=2, Hq=32, Hkv=4, D=128, ps=64, P=100, maxkv=4096, maxsq=512, Tq=600, ks=kp, ws=None)
+    args = dict(B=2, Hq=32, Hkv=4, D=128, ps=64, P=100, maxkv=4096, maxsq=512, Tq=600, ks=kp, ws=None, splits=1)
 
     def call(**kw):
         a = dict(args, **kw)
         return f(fake, fake, fake, fake, None, fake, fake, 64, fake, a["B"], a["maxsq"], a["Tq"], a["Hq"],
                  a["Hkv"], a["D"], a["ps"], a["P"], a["maxkv"], q2, q2, a["ks"], a["ks"],
-                 rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, a["ws"], 1 << 30 if a["ws"] else 0, None)
+                 rsd.ATTN_LSE_PADDED_BSH, 0.088, 1, a["splits"], a["ws"], 1 << 30 if a["ws"] else 0, None)
 
     assert call() == rsd.ATTN_ERR_WORKSPACE                 # the work list needs a workspace
     assert call(D=96) == rsd.ATTN_ERR_UNSUPPORTED
@@ -216,8 +216,22 @@ def test_paged_prefill_rejects_bad_args_on_host(lib):
     # a page stride that is not a whole number of 8-row groups
     assert call(ks=L3(4 * 64 * 128 + 8, 128, 64 * 128)) == rsd.ATTN_ERR_UNSUPPORTED
     assert call(B=0) == rsd.ATTN_OK                          # nothing to do
-    assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 32, 4) == \
+    assert call(splits=0) == rsd.ATTN_ERR_INVALID_ARG
+    assert call(splits=5000) == rsd.ATTN_ERR_INVALID_ARG
+    # without splits the workspace is the prefill work list; with splits it adds the short rows'
+    # partials: B * qmax * Hq rows of D floats and an LSE per split, qmax = min(4, 64 / G, max_seqlen_q)
+    assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 32, 4, 128, 1) == \
         rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 32, 4)
+    base = rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 32, 4)
+    rows = 2 * 4 * 32          # G = 8: qmax = min(4, 8, 512) = 4
+    n3 = rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 32, 4, 128, 3)
+    assert n3 >= base + 3 * rows * 128 * 4 + 3 * rows * 4 + 2 * 4 and n3 % 256 == 0
+    rows = 2 * 1 * 64          # G = 64: qmax = 1
+    assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 64, 1, 64, 2) >= \
+        rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 64, 1) + 2 * rows * 64 * 4
+    # G > 64: no routing, no partials
+    assert rsd.attn_fwd_paged_prefill_workspace_size(2, 512, 600, 128, 1, 64, 2) == \
+        rsd.attn_fwd_ragged_workspace_size(2, 512, 600, 128, 1)
 
 
 def test_sizes_past_the_32_bit_token_range_are_declined(lib):

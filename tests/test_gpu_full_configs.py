@@ -112,7 +112,7 @@ def test_paged_prefill_full_size():
     T, smax = q.shape[0], int(lq.max())
     o = torch.full_like(q, float("nan"))
     lse = torch.full((w.B, smax, w.Hq), float("nan"), dtype=torch.float32, device=DEV)
-    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv), dtype=torch.uint8,
+    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv, w.Dqk, 1), dtype=torch.uint8,
                      device=DEV)
     rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, torch.as_tensor(cu_q, device=DEV),
                                torch.as_tensor(table, device=DEV), torch.as_tensor(kl, device=DEV),
@@ -122,15 +122,28 @@ def test_paged_prefill_full_size():
     assert rsd.attn_get_device_error() == rsd.ATTN_OK
     assert not torch.isnan(o).any()
     rng = np.random.default_rng(2)
-    for b in (0, 7, 15):
+    # every sequence: first and last query row, rows on both sides of each 128-row query tile
+    # boundary and of each page boundary of the query chunk (query i sits at cache position
+    # L - n + i), plus 512 random rows spread over the sequences
+    extra = {b: [] for b in range(w.B)}
+    for _ in range(512):
+        b = int(rng.integers(w.B))
+        extra[b].append(int(rng.integers(int(lq[b]))))
+    n_checked = 0
+    for b in range(w.B):
         L, n = int(kl[b]), int(lq[b])
+        idx = {0, n - 1}
+        for t in range(128, n, 128):
+            idx |= {t - 1, t}
+        first_pos = L - n
+        for pos in range((first_pos // w.page_size + 1) * w.page_size, L, w.page_size):
+            idx |= {pos - 1 - first_pos, pos - first_pos}
+        idx = sorted(i for i in idx | set(extra[b]) if 0 <= i < n)
         j = np.arange(L)
         pages = torch.as_tensor(table[b, j // w.page_size].astype(np.int64), device=DEV)
         slots = torch.as_tensor(j % w.page_size, device=DEV)
         kc, vc = kp[pages, :, slots].contiguous(), vp[pages, :, slots].contiguous()
-        rows = [(0, int(rng.integers(w.Hq)), i) for i in (0, 127, 128, n - 1)]
-        rows += [(0, int(rng.integers(w.Hq)), int(rng.integers(n))) for _ in range(60)]
-        rows = np.array(rows, dtype=np.int32)
+        rows = np.array([(0, int(rng.integers(w.Hq)), i) for i in idx], dtype=np.int32)
         q_b = q[int(cu_q[b]):int(cu_q[b + 1])]
         o_ref, l_ref = orc().attn_ragged_rows(bits(q_b), bits(kc), bits(vc), np.array([0, n]),
                                               np.array([0, L]), w.Hq, w.Hkv, w.scale, True, rows)
@@ -138,3 +151,5 @@ def test_paged_prefill_full_size():
         hh = torch.as_tensor(rows[:, 1].astype(np.int64), device=DEV)
         assert_o_close(o[tok, hh], o_ref, f"paged prefill full b={b}")
         assert_lse_close(lse[b, tok - int(cu_q[b]), hh], l_ref, f"paged prefill full b={b}")
+        n_checked += len(rows)
+    assert n_checked >= 512 + 16 * 2

@@ -115,7 +115,10 @@ def test_paged_prefill_work_list_bit_exact():
     torch.cuda.synchronize()
     assert rsd.attn_get_device_error() == rsd.ATTN_OK
     count, claims, items = _header_items(ws, (n - 256) // 16)
-    mc.check_sequence_list(items, count, np.array(lq), np.array(lkv), Hq, Hkv, True)
+    # the 1-, 2- and 4-query sequences go to the split-KV decode kernel: no prefill items
+    short_q = mc.routed_qmax(Hq // Hkv, max(lq))
+    assert short_q == 4
+    mc.check_sequence_list(items, count, np.array(lq), np.array(lkv), Hq, Hkv, True, short_q)
     n_pairs = Hq // mc.heads_per_item(Hq, Hkv)
     assert claims == count + min(mc.ragged_max_tiles(len(lq), max(lq), T) * n_pairs, _sms())
 

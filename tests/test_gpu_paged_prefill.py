@@ -42,20 +42,21 @@ def _gather(pool, table, lens_kv, ps, layout):
     return torch.cat(parts, 0).contiguous()
 
 
-def _run(q, k, v, table, kl, cu_q, ps, scale, causal, layout="HND", lse_layout=rsd.ATTN_LSE_PADDED_BSH):
+def _run(q, k, v, table, kl, cu_q, ps, scale, causal, layout="HND", lse_layout=rsd.ATTN_LSE_PADDED_BSH,
+         num_splits=1):
     B = len(cu_q) - 1
     max_sq = max(1, int(np.max(np.diff(cu_q))))
-    Hq = q.shape[1]
+    Hq, D = q.shape[1], q.shape[2]
     o = torch.full((q.shape[0], Hq, v.shape[-1]), float("nan"), dtype=torch.bfloat16, device=DEV)
     lse = lse_alloc(lse_layout, B, max_sq, q.shape[0], Hq, float("nan"), DEV)
     Hkv = k.shape[1] if layout == "HND" else k.shape[2]
-    ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(B, max_sq, q.shape[0], Hq, Hkv),
-                     dtype=torch.uint8, device=DEV)
+    ws = torch.full((rsd.attn_fwd_paged_prefill_workspace_size(B, max_sq, q.shape[0], Hq, Hkv, D, num_splits),),
+                    0xFF, dtype=torch.uint8, device=DEV)  # stale partials must be overwritten
     rsd.attn_fwd_paged_prefill(
         q, k, v, o, lse, torch.as_tensor(cu_q, device=DEV), torch.as_tensor(table, device=DEV),
         torch.as_tensor(kl, device=DEV), max_seqlen_q=max_sq, page_size=ps,
         max_kv_len=max(1, int(np.max(kl))), scale=scale, causal=causal, workspace=ws,
-        lse_layout=lse_layout, kv_layout=layout)
+        lse_layout=lse_layout, kv_layout=layout, num_splits=num_splits)
     torch.cuda.synchronize()
     assert rsd.attn_get_device_error() == rsd.ATTN_OK
     return o, lse
@@ -88,6 +89,9 @@ def test_paged_prefill_vs_oracle(lens_q, lens_kv, Hq, Hkv, D, ps, layout, causal
 
 
 def test_paged_prefill_matches_ragged_over_gathered_kv_bitwise():
+    """The sequences on prefill tiles give exactly what the ragged kernel gives
+    over their gathered K/V (the 1-query sequence takes the decode kernel and is
+    checked against the oracle elsewhere)."""
     lens_q, lens_kv, ps = [128, 300, 1], [1024, 300, 777], 64
     q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 16, 4, 128, ps, seed=5)
     o1, l1 = _run(q, k, v, table, kl, cu_q, ps, 0.09, True, lse_layout=rsd.ATTN_LSE_PACKED_TH)
@@ -95,7 +99,8 @@ def test_paged_prefill_matches_ragged_over_gathered_kv_bitwise():
     cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
     o2, l2 = ragged_gpu(q, kc, vc, cu_q, cu_kv, int(max(lens_q)), int(max(lens_kv)), 0.09, True,
                         lse_layout=rsd.ATTN_LSE_PACKED_TH)
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    long_tok = int(cu_q[2])  # tokens of the two prefill sequences
+    assert torch.equal(o1[:long_tok], o2[:long_tok]) and torch.equal(l1[:long_tok], l2[:long_tok])
 
 
 @pytest.mark.parametrize("ps", [16, 64])
@@ -161,3 +166,77 @@ def test_paged_prefill_independent_kv_tables():
     og, lg = gather_ragged(o, lse, cu_q, rows, rsd.ATTN_LSE_PACKED_TH)
     assert_o_close(og, o_ref, "paged prefill, independent tables")
     assert_lse_close(lg, l_ref, "paged prefill, independent tables")
+
+
+# --------------------------------------------------------------------------------------------
+# Mixed batches: sequences of at most qmax = min(4, 64 / G) queries run on the split-KV decode
+# kernel (G heads x Lq tokens as the tile rows), the others on prefill tiles, in one call.
+MIXED = [
+    # (lens_q, lens_kv, Hq, Hkv, D, ps, splits, causal, lse_layout)
+    ([1, 2, 4, 1000, 3], [32768, 20000, 32000, 32768, 5], 8, 2, 128, 64, 1, True, rsd.ATTN_LSE_PADDED_BSH),
+    ([1, 2, 4, 1000, 3], [32768, 20000, 32000, 32768, 5], 8, 2, 128, 64, 4, True,
+     rsd.ATTN_LSE_PACKED_TH | rsd.ATTN_LSE_LOG2),
+    ([1, 2, 4, 500], [9000, 4100, 7000, 3000], 16, 2, 128, 64, 3, True, rsd.ATTN_LSE_PACKED_HT),    # 32 rows
+    ([1, 4, 3, 200], [3000, 5000, 2, 1000], 32, 2, 64, 16, 2, True, rsd.ATTN_LSE_PADDED_BSH),      # 64 rows
+    ([1, 2, 2, 300], [4000, 1000, 64, 2000], 32, 1, 128, 32, 5, True, rsd.ATTN_LSE_PACKED_TH),     # G 32
+    ([1, 3, 4, 130], [1000, 999, 4097, 130], 6, 2, 64, 128, 2, False, rsd.ATTN_LSE_PADDED_BSH),    # G 3
+    ([1] * 8 + [4] * 8, [100 * i + 1 for i in range(16)], 8, 2, 128, 64, 3, True, rsd.ATTN_LSE_PACKED_TH),
+]
+
+
+@pytest.mark.parametrize("lens_q,lens_kv,Hq,Hkv,D,ps,splits,causal,lse_layout", MIXED)
+def test_mixed_batch_every_row_vs_oracle(lens_q, lens_kv, Hq, Hkv, D, ps, splits, causal, lse_layout):
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, Hq, Hkv, D, ps, seed=Hq + splits + len(lens_q))
+    scale = 1.0 / np.sqrt(D)
+    o, lse = _run(q, k, v, table, kl, cu_q, ps, scale, causal, lse_layout=lse_layout, num_splits=splits)
+    kc, vc = _gather(k, table, kl, ps, "HND"), _gather(v, table, kl, ps, "HND")
+    cu_kv = np.concatenate([[0], np.cumsum(kl)]).astype(np.int32)
+    rows = ragged_rows_all(cu_q, Hq)
+    o_ref, l_ref = orc().attn_ragged_rows(bits(q), bits(kc), bits(vc), cu_q, cu_kv, Hq, Hkv, scale, causal, rows)
+    og, lg = gather_ragged(o, lse, cu_q, rows, lse_layout)
+    where = f"mixed batch {lens_q} G={Hq // Hkv} splits={splits}"
+    assert_o_close(og, o_ref, where)
+    if lse_layout & rsd.ATTN_LSE_LOG2:
+        assert_lse_close(lg, l_ref * LOG2E, where, atol=LSE_ATOL * LOG2E)
+    else:
+        assert_lse_close(lg, l_ref, where)
+    if (lse_layout & ~rsd.ATTN_LSE_LOG2) == rsd.ATTN_LSE_PADDED_BSH:
+        for b, n in enumerate(lens_q):  # padded rows past each length stay -inf
+            assert torch.all(lse[b, n:] == -float("inf"))
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+def test_single_query_rows_equal_paged_decode_bitwise(splits):
+    """A 1-query sequence in a mixed batch (G = 4: one m16 tile) is computed
+    exactly as attn_fwd_paged computes a decode row with the same splits."""
+    lens_q, lens_kv, ps, Hq, Hkv, D = [1, 1, 1, 700], [5000, 64, 1, 3000], 64, 8, 2, 128
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, Hq, Hkv, D, ps, seed=31)
+    o, lse = _run(q, k, v, table, kl, cu_q, ps, 0.088, True, lse_layout=rsd.ATTN_LSE_PACKED_TH,
+                  num_splits=splits)
+    n = 3
+    qd = q[:n].contiguous()
+    od = torch.full((n, Hq, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    ld = torch.full((n, Hq), float("nan"), dtype=torch.float32, device=DEV)
+    wsn = rsd.attn_fwd_paged_workspace_size(n, Hq, D, splits)
+    ws = torch.empty(max(wsn, 1), dtype=torch.uint8, device=DEV) if wsn else None
+    rsd.attn_fwd_paged(qd, k, v, od, ld, torch.as_tensor(table[:n], device=DEV), torch.as_tensor(kl[:n], device=DEV),
+                       page_size=ps, max_kv_len=int(max(lens_kv)), scale=0.088, num_splits=splits, workspace=ws)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    assert torch.equal(o[:n], od) and torch.equal(lse[:n], ld)
+
+
+def test_mixed_batch_nan_past_kv_len_in_short_rows():
+    """NaN in the unused slots of the last page of short (decode-kernel) sequences never reaches O."""
+    lens_q, lens_kv, ps = [1, 3, 200], [170, 90, 333], 64
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=41)
+    kn, vn = k.clone(), v.clone()
+    for b, L in enumerate(lens_kv):
+        last = table[b, (L - 1) // ps]
+        kn[last, :, L % ps:] = float("nan")
+        vn[last, :, L % ps:] = float("nan")
+    for splits in (1, 2):
+        o1, l1 = _run(q, k, v, table, kl, cu_q, ps, 0.1, True, num_splits=splits)
+        o2, l2 = _run(q, kn, vn, table, kl, cu_q, ps, 0.1, True, num_splits=splits)
+        assert torch.isfinite(o2.float()).all()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)

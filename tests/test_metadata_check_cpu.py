@@ -95,3 +95,18 @@ def test_page_coords_rule():
     table = np.array([[7, 2, -1], [0, 9, 1]], dtype=np.int32)
     got = mc.page_coords(table, [0, 0, 1, 0, 1], [0, 70, 65, 130, 127], 64, 9, 8)
     assert got.tolist() == [[7, 0, 56], [2, 6, 16], [-1, 1, -1], [-1, 2, -1], [-1, 63, -1]]
+
+
+def test_routed_short_sequences_have_no_items():
+    lq = np.array([1, 4, 5, 0, 300], dtype=np.int64)
+    lkv = np.array([900, 100, 5, 3, 300], dtype=np.int64)
+    assert mc.routed_qmax(4, 300) == 4 and mc.routed_qmax(32, 300) == 2 and mc.routed_qmax(128, 300) == 0
+    assert mc.sequence_block(0, 1, 900, 8, 2, True, short_q=4) == []
+    keys = [mc.sequence_key(int(a), int(b), True, 4) for a, b in zip(lq, lkv)]
+    order = sorted(range(len(lq)), key=lambda b: -keys[b])
+    items = [it for b in order for it in mc.sequence_block(b, int(lq[b]), int(lkv[b]), 8, 2, True, 4)]
+    mc.check_sequence_list(np.array(items), len(items), lq, lkv, 8, 2, True, short_q=4)
+    # a list that still holds the 1-query sequence's items is rejected
+    extra = mc.sequence_block(0, 1, 900, 8, 2, True)
+    with pytest.raises(AssertionError):
+        mc.check_sequence_list(np.array(items + extra), len(items) + len(extra), lq, lkv, 8, 2, True, short_q=4)
