@@ -39,15 +39,16 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes (read + write) from the latest ncu capture of each kernel on its
 # small case, as a ratio to the bytes that scale with the launch, applied to
-# the full launch.  None when the kernel changed after the counters were taken.
-#   paged_decode: per K/V byte, batch 32 (2.686 / 2.673 GB)
-#   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.041 / 1.061 GB)
-#   mla_decode: per K/V byte, batch 8 (0.346 / 0.335 GB; the partials grow with the
+# the full launch.  None when the kernel changed after the counters were taken
+# or has no capture.
+#   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.0404 / 1.0611 GB)
+#   paged_decode: per K/V byte, batch 32 (2.6866 / 2.6734 GB)
+#   mla_decode: per K/V byte, batch 8 (0.3439 / 0.3355 GB; the partials grow with the
 #     batch like the K/V bytes)
 #   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.683 / 0.635 GB)
-#   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (1.049 / 0.671 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9807, "paged_decode": 1.0048, "mla_decode": 1.0307, "paged_prefill": 1.0764,
-                 "dense_prefill": 1.5627}
+#   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7045 / 0.6711 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0251, "paged_prefill": 1.0764,
+                 "dense_prefill": 1.0497}
 
 
 def load_peaks():
@@ -659,10 +660,24 @@ def run_ours(args):
 
     cpu = {}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        orc = oracle.default()
+        all_cores = orc.num_threads()
         v, c, desc = oracle_prefill_sample(pdata, args.cpu_seconds)
         cpu["prefill"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": c, "kind": "oracle", "sample": desc}
         v, c, desc = oracle_decode_sample(ddata, args.cpu_seconds)
         cpu["decode"] = {"value": round(v, 4), "unit": "GB/s", "cores": c, "kind": "oracle", "sample": desc}
+        # the same oracle on one core, on a smaller bounded sample
+        orc.set_num_threads(1)
+        try:
+            v, c, desc = oracle_prefill_sample(pdata, args.cpu_seconds / 3)
+            cpu["prefill_single_core"] = {"value": round(v, 7), "unit": "TFLOP/s", "cores": c, "kind": "oracle",
+                                          "sample": desc}
+            v, c, desc = oracle_decode_sample(ddata, args.cpu_seconds / 3)
+            cpu["decode_single_core"] = {"value": round(v, 5), "unit": "GB/s", "cores": c, "kind": "oracle",
+                                         "sample": desc}
+        finally:
+            orc.set_num_threads(all_cores)
 
     extra_out = {}
     for part in extras:
@@ -710,7 +725,9 @@ def run_ours(args):
                        "samples": ck["samples"]},
         }
         if cpu:
-            line["cpu_baseline"] = dict(cpu["prefill"], decode=cpu["decode"])
+            line["cpu_baseline"] = dict(cpu["prefill"], decode=cpu["decode"],
+                                        single_core={"prefill": cpu.get("prefill_single_core"),
+                                                     "decode": cpu.get("decode_single_core")})
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -91,6 +91,10 @@ class Oracle:
     def num_threads(self) -> int:
         return int(self._lib.oracle_num_threads())
 
+    def set_num_threads(self, n: int) -> None:
+        """Threads the oracle's OpenMP loops use from now on (threading only)."""
+        self._lib.oracle_set_num_threads(ctypes.c_int(int(n)))
+
     def attn_ragged_rows(self, q, k, v, cu_q, cu_kv, Hq, Hkv, scale, causal, rows,
                          q_strides=None, k_strides=None, v_strides=None):
         """Rows (b, h, i) of ragged/THD attention, i the query index in its sequence.

@@ -264,3 +264,15 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* Sets the threads OpenMP uses from now on (the CPU baseline times the oracle
+ * on all cores and on one).  Threading only: the arithmetic is unchanged. */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    omp_set_num_threads(n > 0 ? n : 1);
+#else
+    (void)n;
+#endif
+}

@@ -174,10 +174,13 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
 // processing time first: the last items claimed are the cheapest), and inside
 // a group (batch, kv head, query tile longest first, head pair), so the CTAs
 // working at the same time read few (batch, kv head) K/V streams and each
-// stream's prefix is brought from HBM once per group.  Grid-stride over the
+// stream's causal prefix is brought from HBM once per group.  On the dense
+// workload (B 8, S 4096) groups of 16 read K/V 1.5 times from HBM (1.05x the
+// algorithmic bytes in all) against 2.5 times with groups of 8, at the same
+// speed.  Grid-stride over the
 // items; block 0 writes the header.
 // ---------------------------------------------------------------------------
-constexpr int kDenseQtGroup = 8;
+constexpr int kDenseQtGroup = 16;
 
 __global__ void __launch_bounds__(256) dense_worklist_kernel(int B, int Sq, int Skv, int causal, int Hkv,
                                                              int pairs_per_group, int heads_per_item, int G,

@@ -14,7 +14,7 @@ head h0 of the pair, KV tiles the item visits)):
     short_q = min(4, 64 / G, max_seqlen_q)); a sequence's items form one contiguous run ordered
     (kv head, query tile longest first, head pair); runs are ordered by the
     sequence's total tile steps (capped at 4095), most first, ties in any order;
-  * dense: groups of 8 query tiles, the group of longest tiles first, inside a
+  * dense: groups of 16 query tiles, the group of longest tiles first, inside a
     group (batch, kv head, query tile longest first, head pair);
   * header[0] = item count; after the prefill ran, header[1] = item count +
     number of persistent CTAs (each CTA makes one claim past the end).
@@ -24,7 +24,7 @@ from __future__ import annotations
 import numpy as np
 
 SORT_CAP = 4095
-DENSE_GROUP = 8
+DENSE_GROUP = 16
 
 
 def heads_per_item(Hq, Hkv):
