@@ -45,9 +45,9 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 #   paged_decode: per K/V byte, batch 32 (2.6866 / 2.6734 GB)
 #   mla_decode: per K/V byte, batch 8 (0.3439 / 0.3355 GB; the partials grow with the
 #     batch like the K/V bytes)
-#   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.683 / 0.635 GB)
+#   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.6837 / 0.6345 GB)
 #   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7045 / 0.6711 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0251, "paged_prefill": 1.0764,
+TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0251, "paged_prefill": 1.0776,
                  "dense_prefill": 1.0497}
 
 
@@ -101,6 +101,9 @@ class ClockSampler:
         self.proc = None
         self.nvml = None
         self.lines = []
+        # samples are kept only while a part is being timed (not in the idle gaps
+        # between parts, whose clocks say nothing about the measurement)
+        self.active = False
 
     def __enter__(self):
         try:
@@ -112,7 +115,7 @@ class ClockSampler:
             self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
             self.nvml = pynvml
             self._stop = threading.Event()
-            self._sample_nvml()  # one sample before the timing starts
+            self._sample_nvml(force=True)  # one sample before the timing starts
             self._t = threading.Thread(target=self._loop_nvml, daemon=True)
             self._t.start()
             return self
@@ -129,7 +132,9 @@ class ClockSampler:
             self.proc = None
         return self
 
-    def _sample_nvml(self):
+    def _sample_nvml(self, force=False):
+        if not (self.active or force):
+            return
         n, h = self.nvml, self.handle
         sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
         mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
@@ -147,7 +152,8 @@ class ClockSampler:
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            if self.active:
+                self.lines.append(ln.strip())
 
     def __exit__(self, *a):
         if self.nvml is not None:
@@ -612,8 +618,16 @@ def run_ours(args):
 
     results = {}
     with ClockSampler(local) as clocks:
-        for part in [prefill, decode] + extras:
+        for i, part in enumerate([prefill, decode] + extras):
+            if i > 0 and args.part_gap > 0:
+                # every part starts from an idle GPU: the power state one part leaves
+                # behind would otherwise carry into the next (the dense prefill measured
+                # ~12 % slower right after the ragged prefill than after 2 s idle)
+                torch.cuda.synchronize()
+                time.sleep(args.part_gap)
+            clocks.active = True
             total_ms, per = time_part(torch, part, args.steps, args.warmup, dist, world)
+            clocks.active = False
             results[part.name] = (total_ms, per)
     assert rsd.attn_get_device_error() == rsd.ATTN_OK, "device-side error during the bench"
 
@@ -812,6 +826,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--part-gap", type=float, default=2.0,
+                    help="seconds of idle GPU before each part after the first")
     ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "paged_prefill",
                                        "mla_decode", "mixed_batch", "mixed_short_rows", "mixed_chunks"],
                     help="profiling: time one part only and print its own line")

@@ -253,3 +253,13 @@ def test_sizes_past_the_32_bit_token_range_are_declined(lib):
     kp = L3(8 * 64 * 128, 128, 64 * 128)
     assert g(fake, fake, fake, fake, None, fake, 64, fake, 65536, 64, 8, 128, 128, 64, 100, 4096,
              q2, q2, kp, kp, 0.088, 1, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED   # B > 65535
+
+
+def test_page_coords_diagnostic_rejects_bad_args_on_host(lib):
+    f = lib.attn_selftest_page_coords
+    fake = ctypes.c_void_p(0x100000)
+    assert f(fake, 64, 64, 100, 8, fake, fake, 0, fake, None) == rsd.ATTN_OK          # nothing to do
+    assert f(fake, 64, 0, 100, 8, fake, fake, 5, fake, None) == rsd.ATTN_ERR_INVALID_ARG   # page size 0
+    assert f(fake, 64, 64, 0, 8, fake, fake, 5, fake, None) == rsd.ATTN_ERR_INVALID_ARG    # no pages
+    assert f(None, 64, 64, 100, 8, fake, fake, 5, fake, None) == rsd.ATTN_ERR_INVALID_ARG  # no table
+    assert f(fake, 64, 64, 1 << 30, 8, fake, fake, 5, fake, None) == rsd.ATTN_ERR_UNSUPPORTED  # groups >= 2^31
