@@ -181,6 +181,8 @@ MIXED = [
     ([1, 2, 2, 300], [4000, 1000, 64, 2000], 32, 1, 128, 32, 5, True, rsd.ATTN_LSE_PACKED_TH),     # G 32
     ([1, 3, 4, 130], [1000, 999, 4097, 130], 6, 2, 64, 128, 2, False, rsd.ATTN_LSE_PADDED_BSH),    # G 3
     ([1] * 8 + [4] * 8, [100 * i + 1 for i in range(16)], 8, 2, 128, 64, 3, True, rsd.ATTN_LSE_PACKED_TH),
+    # short rows over an empty cache and a 1-key cache (the first query of the 2 sees no key)
+    ([1, 2, 300, 4], [0, 1, 500, 70], 8, 2, 128, 64, 2, True, rsd.ATTN_LSE_PADDED_BSH),
 ]
 
 
