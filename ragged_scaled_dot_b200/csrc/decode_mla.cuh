@@ -13,9 +13,10 @@
 //
 //   rank 0, the score CTA: S = Q K^T (N = R keys per page box, K = 576; all of
 //     Q sits in TMEM as the A operand), then the online softmax.  P (bf16,
-//     128 x 64), the per-row rescale factors and, with the last chunk, 1/l go
-//     to rank 1 as one message: a bulk copy from a staging buffer into rank
-//     1's shared memory that completes on rank 1's mbarrier.
+//     128 x 64), the per-row rescale factors and 1/l (read with the last
+//     chunk) go to rank 1 as one message: the softmax threads store it
+//     straight into rank 1's shared memory with st.async, every store
+//     counting its bytes on rank 1's mbarrier.
 //   rank 1, the value CTA: O += P V in four 128-column quarters (N = 128,
 //     K = 64 keys), O in TMEM; rescales O rows when a message asks for it;
 //     writes O / 1/l (or the fp32 split partial).
@@ -48,7 +49,7 @@ struct MlaTcCfg {
     static constexpr int KLOADS = 9 / KB, VLOADS = 8 / VB;  // loads per chunk
     static constexpr uint32_t KSLOT = KB * BLK;          // [page][KB blocks][R rows][128 B]
     static constexpr uint32_t VSLOT = VB * BLK;          // [page][VB blocks][R rows][128 B]
-    static constexpr int RK = 2;                         // score CTA ring (loads in flight)
+    static constexpr int RK = 3;                         // score CTA ring (loads in flight)
     static constexpr int RV = 2;                         // value CTA ring
     static constexpr uint32_t P_TILE = 128u * 128u;      // P: 128 heads x 64 keys bf16, 128B swizzle
     static constexpr uint32_t MSG_ALPHA = P_TILE;        // float[128] rescale factor per row
@@ -56,10 +57,9 @@ struct MlaTcCfg {
     static constexpr uint32_t MSG_HDR = MSG_INVL + 512;    // int[4]: flags (1 rescale, 2 last), chunk
     static constexpr uint32_t MSG_BYTES = MSG_HDR + 16;
     static constexpr uint32_t PSLOT = 18u * 1024u;       // one message slot, 1024-aligned
-    // score CTA
+    // score CTA: the K ring only (messages are stored straight into the value CTA's slots)
     static constexpr uint32_t S_RING = 0;
-    static constexpr uint32_t S_STAGE = RK * KSLOT;      // two outgoing message buffers
-    static constexpr uint32_t S_END = S_STAGE + 2 * PSLOT;
+    static constexpr uint32_t S_END = RK * KSLOT;
     // value CTA
     static constexpr uint32_t V_RING = 0;
     static constexpr uint32_t V_P = RV * VSLOT;          // two incoming message slots
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
                     a0 = fmin3(a0, a1, fminf(a2, a3));
                 }
                 xmax[hf * 128 + r] = a0;
-                // the staging buffer of this parity is free once the value CTA released chunk j-2
+                // the value CTA's message slot of this parity is free once it released chunk j-2
                 if (tid == 0)
                     okt = mbar_wait<true>(sBar + C::B_PFREE + 8 * ps, ((j >> 1) & 1) ^ 1, abort_flag) && okt;
                 if (!bar_and(1, C::NW, okt)) break;
@@ -360,8 +360,11 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
                     m_use = m_new;
                 }
                 const bool need = (j > 0) && old_finite && (alpha != 1.f);
-                uint8_t* stg = sgen + C::S_STAGE + ps * C::PSLOT;
-                if (hf == 0) *reinterpret_cast<float*>(stg + C::MSG_ALPHA + 4 * r) = alpha;
+                // the message goes straight into the value CTA's slot ps: every store counts its
+                // bytes on that CTA's barrier (17424 bytes per message, 1/l included every time)
+                const uint32_t slot = peer_slot0 + (uint32_t)ps * C::PSLOT;
+                const uint32_t pbar = peer_pfull0 + 8u * (uint32_t)ps;
+                if (hf == 0) st_async_peer_b32(slot + C::MSG_ALPHA + 4u * r, __float_as_uint(alpha), pbar);
                 const float mref = (m_use == -INFINITY) ? 0.f : m_use;
                 const float2 sc2 = make_float2(sl2, sl2);
                 const float2 nm2 = make_float2(-mref, -mref);
@@ -383,34 +386,30 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
                     pk[e] = pack_bf16(pv.x, pv.y);
                 }
                 // keys 32hf .. 32hf+31: 16-byte chunks 4hf .. 4hf+3 of row r (128B swizzle)
-                uint8_t* rowp = stg + r * 128;
+                const uint32_t rowp = slot + (uint32_t)r * 128u;
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                     const int chunk = 4 * hf + v;
-                    *reinterpret_cast<uint4*>(rowp + ((chunk ^ (r & 7)) << 4)) =
-                        make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    st_async_peer_v4(rowp + (uint32_t)((chunk ^ (r & 7)) << 4),
+                                     make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]), pbar);
                 }
                 l = l * alpha + ((sum0.x + sum0.y) + (sum1.x + sum1.y));
                 const bool last = (j == n_chunks - 1);
+                float invl = 0.f;  // read by the value CTA with the last message only
                 if (last) {
                     // 1/l of the whole row: the two halves exchange their partial sums
                     xsum[hf * 128 + r] = l;
                     bar_and(1, C::NW, true);
                     const float lt = l + xsum[(hf ^ 1) * 128 + r];
-                    if (hf == 0) *reinterpret_cast<float*>(stg + C::MSG_INVL + 4 * r) = (lt > 0.f) ? 1.f / lt : 0.f;
+                    invl = (lt > 0.f) ? 1.f / lt : 0.f;
                     l = lt;
                 }
-                fence_proxy_async_smem();
+                if (hf == 0) st_async_peer_b32(slot + C::MSG_INVL + 4u * r, __float_as_uint(invl), pbar);
                 const bool any = bar_or(1, C::NW, need);
                 if (tid == 0) {
-                    volatile int* hdr = reinterpret_cast<volatile int*>(stg + C::MSG_HDR);
-                    hdr[0] = (any ? 1 : 0) | (last ? 2 : 0);
-                    hdr[1] = j;
-                    fence_proxy_async_smem();
-                    const uint32_t bar = peer_pfull0 + 8u * (uint32_t)ps;
-                    mbar_arrive_expect_tx_peer_relaxed(bar, C::MSG_BYTES);
-                    bulk_copy_to_peer(peer_slot0 + (uint32_t)ps * C::PSLOT, sb + C::S_STAGE + ps * C::PSLOT,
-                                      C::MSG_BYTES, bar);
+                    mbar_arrive_expect_tx_peer_relaxed(pbar, C::MSG_BYTES);
+                    st_async_peer_v4(slot + C::MSG_HDR, make_uint4((any ? 1u : 0u) | (last ? 2u : 0u), (uint32_t)j, 0u, 0u),
+                                     pbar);
                 }
             }
             if (hv && hf == 0) {

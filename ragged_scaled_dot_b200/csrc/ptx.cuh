@@ -155,6 +155,22 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t
         : "memory");
 }
 
+// Asynchronous stores into a peer CTA's shared memory (cluster window address)
+// whose bytes count toward the transaction count of the peer's mbarrier, like
+// a bulk copy: the peer's barrier completes when all expected bytes arrived.
+__device__ __forceinline__ void st_async_peer_v4(uint32_t dst_cluster, uint4 v, uint32_t cluster_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+            dst_cluster),
+        "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(cluster_bar)
+        : "memory");
+}
+__device__ __forceinline__ void st_async_peer_b32(uint32_t dst_cluster, uint32_t v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst_cluster),
+                 "r"(v), "r"(cluster_bar)
+                 : "memory");
+}
+
 // Named-barrier reductions over `count` threads (a multiple of 32, every
 // thread of each participating warp): all wait, all get the AND / OR.
 __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool v) {
