@@ -762,13 +762,14 @@ int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_k
     int64_t s_balance;
     double max_overhead;
     if (mla) {
-        // a cluster of two CTAs (one per SM) per (sequence, split, 128-head group): about three
-        // waves of work units over the SM pairs (the launch order puts the longest sequences
-        // first, so few waves suffice; measured best on the 64-sequence MLA workload against
-        // 1, 2, 4 and 5), partial traffic up to ~10% of the KV bytes
+        // a cluster of two CTAs (one per SM) per (sequence, split, 128-head group): about two and
+        // a half waves of work units over the SM pairs (the launch order puts the longest
+        // sequences first, so few waves suffice; on the 64-sequence MLA workload 3 splits measured
+        // 2716 GB/s against 2650-2690 with 4 and 2678 with 2), partial traffic up to ~10% of the
+        // KV bytes
         const int64_t units_per_split = (int64_t)B * ((Hq + 127) / 128);
         const int64_t pairs = num_sms / 2 > 0 ? num_sms / 2 : 1;
-        s_balance = (3 * pairs + units_per_split - 1) / units_per_split;
+        s_balance = (5 * pairs + 2 * units_per_split - 1) / (2 * units_per_split);
         max_overhead = 0.10;
     } else {
         const int64_t ctas_per_split = (int64_t)Hkv * B;
