@@ -260,7 +260,7 @@ def make_ragged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
             "flop_per_unit": "4*D per visible (query, key) pair per query head",
             "traffic_basis_gb": io_gb}
     data = dict(q=q, k=k, v=v, cu=cu, L=L, w=w)
-    return Part("ragged_prefill", "TFLOP/s", flops / 1e12, 3, step, e2e_setup, info), data
+    return Part("ragged_prefill", "TFLOP/s", flops / 1e12, 2, step, e2e_setup, info), data
 
 
 def make_dense_prefill(torch, rsd, synth, dev, seed_offset, B=0):
@@ -306,7 +306,7 @@ def make_paged_prefill(torch, rsd, synth, dev, seed_offset, B=0):
             "kv_tokens": int(L.sum()), "total_pages": int(kp.shape[0]), "traffic_basis_gb": io_gb}
     # padded-LSE fill, the short-row decode kernel (its blocks leave at once: every
     # sequence here has 1024 queries), the work list and the prefill kernel
-    return Part("paged_prefill", "TFLOP/s", flops / 1e12, 4, step, None, info), None
+    return Part("paged_prefill", "TFLOP/s", flops / 1e12, 3, step, None, info), None
 
 
 def make_mixed(torch, rsd, synth, dev, seed_offset, num_sms, subset="all"):

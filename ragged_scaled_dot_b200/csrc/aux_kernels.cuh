@@ -53,12 +53,77 @@ __device__ __forceinline__ int seq_cost_key(int lq, int lk, int causal) {
 // (short_q = 0: the prefill kernel takes every sequence).
 __device__ __forceinline__ int prefill_qtiles(int lq, int short_q) { return lq <= short_q ? 0 : (lq + 127) >> 7; }
 
+// Exclusive prefix sum of v over the block (blockDim.x a multiple of 32, at
+// most 1024); *total gets the block's sum.  warp_sums: 32 ints of shared memory.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += u;
+    }
+    if (lane == 31) warp_sums[wid] = incl;
+    __syncthreads();
+    if (wid == 0) {
+        int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += u;
+        }
+        warp_sums[lane] = w;  // inclusive prefix over warps
+    }
+    __syncthreads();
+    const int out = incl - v + (wid > 0 ? warp_sums[wid - 1] : 0);
+    *total = warp_sums[(blockDim.x >> 5) - 1];
+    __syncthreads();  // warp_sums may be reused after this
+    return out;
+}
+
+// Padded (b, s_max, h) LSE: rows at or past a sequence's length are -inf
+// ("cuDNN Frontend v1.30.0 Release Notes", "New: the FlashInfer serving path
+// runs on FROST": the padded Stats buffer is seeded with -inf on the launch
+// stream).  Rows inside a sequence are written by the attention kernels.
+__device__ __forceinline__ void lse_padded_fill(const int32_t* __restrict__ cu_q, int B, int smax, int Hq,
+                                                float* __restrict__ lse, int64_t warp_id, int64_t n_warps) {
+    // warp w takes rows [w * per, (w + 1) * per) of the B * smax rows; within one
+    // sequence the padded rows are contiguous, so the lanes write that span flat
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)B * smax;
+    const int64_t per = (rows + n_warps - 1) / n_warps;
+    int64_t r = warp_id * per;
+    const int64_t r_end = min(rows, r + per);
+    if (r >= r_end) return;
+    int b = (int)(r / smax);
+    int64_t row0 = (int64_t)b * smax;  // first row of sequence b
+    while (r < r_end) {
+        int lq = cu_q[b + 1] - cu_q[b];
+        lq = max(0, min(lq, smax));
+        const int64_t seg_end = min(r_end, row0 + smax);
+        for (int64_t i = max(r, row0 + lq) * Hq + lane; i < seg_end * Hq; i += 32) lse[i] = -INFINITY;
+        r = seg_end;
+        row0 += smax;
+        ++b;
+    }
+}
+
+// Block 0 builds the list (1024 threads).  Blocks 1.. (when lse is given) write
+// the padded LSE rows past each sequence's length, which the prefill kernel
+// never touches, so the two parts need no ordering.
 __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ cu_kv,
     const int32_t* __restrict__ kv_lens, int B, int max_sq,
     int max_skv, int64_t total_q, int64_t total_kv, int causal, int Hkv, int pairs_per_group,
     int heads_per_item, int G, int* __restrict__ header, int4* __restrict__ items,
-    int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles, int short_q) {
+    int* __restrict__ sorted_nqt, int* __restrict__ rank_of, int max_tiles, int short_q,
+    float* __restrict__ lse, int lse_smax, int Hq) {
+    if (blockIdx.x > 0) {
+        if (lse != nullptr)
+            lse_padded_fill(cu_q, B, lse_smax, Hq, lse, ((int64_t)(blockIdx.x - 1) * blockDim.x + threadIdx.x) >> 5,
+                            ((int64_t)(gridDim.x - 1) * blockDim.x) >> 5);
+        return;
+    }
     __shared__ int hist[kSortBuckets];
     __shared__ int warp_sums[32];
     __shared__ int n_tiles_sh;
@@ -83,10 +148,17 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         atomicAdd(&n_tiles_sh, nqt);
     }
     __syncthreads();
-    // 2. bucket starts, largest count first (one thread: 4096 buckets)
-    if (tid == 0) {
-        int run = 0;
-        for (int c = kSortBuckets - 1; c >= 0; --c) {
+    // 2. bucket starts, largest key first: thread t owns positions
+    //    [t * per, (t + 1) * per) of the buckets in descending key order
+    {
+        const int per = (kSortBuckets + blockDim.x - 1) / blockDim.x;
+        const int p0 = min(kSortBuckets, tid * per), p1 = min(kSortBuckets, p0 + per);
+        int local = 0;
+        for (int pos = p0; pos < p1; ++pos) local += hist[kSortBuckets - 1 - pos];
+        int total;
+        int run = block_exclusive_scan(local, warp_sums, &total);
+        for (int pos = p0; pos < p1; ++pos) {
+            const int c = kSortBuckets - 1 - pos;
             const int h = hist[c];
             hist[c] = run;
             run += h;
@@ -106,35 +178,18 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
     }
     __syncthreads();
     // exclusive scan of sorted_nqt (in place), chunked over the block
-    const int per = (B + blockDim.x - 1) / blockDim.x;
-    const int lo = min(B, tid * per), hi = min(B, lo + per);
-    int local = 0;
-    for (int i = lo; i < hi; ++i) local += sorted_nqt[i];
-    // block-wide exclusive scan of `local`
-    int incl = local;
-    const int lane = tid & 31, wid = tid >> 5;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_sums[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int w = (lane < (int)(blockDim.x >> 5)) ? warp_sums[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += v;
+    {
+        const int per = (B + blockDim.x - 1) / blockDim.x;
+        const int lo = min(B, tid * per), hi = min(B, lo + per);
+        int local = 0;
+        for (int i = lo; i < hi; ++i) local += sorted_nqt[i];
+        int total;
+        int run = block_exclusive_scan(local, warp_sums, &total);
+        for (int i = lo; i < hi; ++i) {
+            const int v = sorted_nqt[i];
+            sorted_nqt[i] = run;
+            run += v;
         }
-        warp_sums[lane] = w;  // inclusive prefix over warps
-    }
-    __syncthreads();
-    int run = incl - local + (wid > 0 ? warp_sums[wid - 1] : 0);
-    for (int i = lo; i < hi; ++i) {
-        const int v = sorted_nqt[i];
-        sorted_nqt[i] = run;
-        run += v;
     }
     __syncthreads();
     const int n_tiles = min(n_tiles_sh, max_tiles);
@@ -143,9 +198,11 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         header[0] = n_tiles * (Hkv * pairs_per_group);
         header[1] = 0;
     }
-    // 3. items of each sequence: (kv head, query tile longest first, head pair)
+    // 3. items of each sequence, one warp per sequence: (kv head, query tile
+    //    longest first, head pair)
     const int n_pairs = Hkv * pairs_per_group;
-    for (int b = tid; b < B; b += blockDim.x) {
+    const int lane = tid & 31, nwarps = blockDim.x >> 5;
+    for (int b = tid >> 5; b < B; b += nwarps) {
         if (!ragged_seq_ok(cu_q, cu_kv, kv_lens, b, max_sq, max_skv, total_q, total_kv)) continue;
         const int lq = cu_q[b + 1] - cu_q[b], lk = seq_kv_len(cu_kv, kv_lens, b);
         const int nqt = prefill_qtiles(lq, short_q);
@@ -153,15 +210,15 @@ __global__ void __launch_bounds__(1024) ragged_worklist_kernel(
         const int tile0 = sorted_nqt[rank_of[b]];  // first tile slot of this sequence
         if (tile0 + nqt > max_tiles) continue;
         const int64_t base = (int64_t)tile0 * n_pairs;
-        for (int g = 0; g < Hkv; ++g)
-            for (int t = 0; t < nqt; ++t) {
-                const int qt = nqt - 1 - t;
-                const int cost = prefill_n_kv(qt, lq, lk, causal);
-                for (int pr = 0; pr < pairs_per_group; ++pr) {
-                    const int64_t idx = base + ((int64_t)g * nqt + t) * pairs_per_group + pr;
-                    items[idx] = make_int4(b, qt, g * G + pr * heads_per_item, cost);
-                }
-            }
+        const int per_g = nqt * pairs_per_group;
+        for (int i = lane; i < Hkv * per_g; i += 32) {
+            const int g = i / per_g;
+            const int rem = i - g * per_g;
+            const int t = rem / pairs_per_group;
+            const int pr = rem - t * pairs_per_group;
+            const int qt = nqt - 1 - t;
+            items[base + i] = make_int4(b, qt, g * G + pr * heads_per_item, prefill_n_kv(qt, lq, lk, causal));
+        }
     }
 }
 
@@ -270,24 +327,6 @@ __global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restri
     }
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) order[atomicAdd(&hist[bucket(b)], 1)] = b;
-}
-
-// Padded (b, s_max, h) LSE: rows at or past a sequence's length are -inf
-// ("cuDNN Frontend v1.30.0 Release Notes", "New: the FlashInfer serving path
-// runs on FROST": the padded Stats buffer is seeded with -inf on the launch
-// stream).  Rows inside a sequence are written by the prefill kernel.
-__global__ void lse_padded_fill_kernel(const int32_t* __restrict__ cu_q, int B, int smax, int Hq,
-                                       float* __restrict__ lse) {
-    const int64_t n = (int64_t)B * smax * Hq;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t bs = i / Hq;
-        const int b = (int)(bs / smax);
-        const int s = (int)(bs - (int64_t)b * smax);
-        int lq = cu_q[b + 1] - cu_q[b];
-        lq = max(0, min(lq, smax));
-        if (s >= lq) lse[i] = -INFINITY;
-    }
 }
 
 // ---------------------------------------------------------------------------

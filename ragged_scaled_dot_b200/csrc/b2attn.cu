@@ -144,6 +144,15 @@ bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
 int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
 
+// Extra blocks of the work-list launch that write the padded LSE rows past
+// each sequence's length: 0 unless the LSE is in the padded (b, s_max, h)
+// layout; at most two 1024-thread blocks per SM.
+int lse_fill_blocks(const float* lse, int lse_base, int B, int smax, int Hq, int sms) {
+    if (lse == nullptr || lse_base != ATTN_LSE_PADDED_BSH) return 0;
+    const int64_t want = ((int64_t)B * smax * Hq + 1023) / 1024;
+    return (int)(want < (int64_t)sms * 2 ? want : (int64_t)sms * 2);
+}
+
 // A stride for a tensor-map dimension of extent 1 (never stepped along).
 int64_t unit_dim_stride(int64_t a, int64_t b) { return round_up(a > b ? a : b, 8); }
 
@@ -440,17 +449,12 @@ int attn_fwd_ragged(const void* q, const void* k, const void* v, void* o, float*
     int* header = reinterpret_cast<int*>(wsb);
     int4* items = reinterpret_cast<int4*>(wsb + wl.items_off);
 
-    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
+    const int fill = lse_fill_blocks(lse, lse_base, B, max_seqlen_q, Hq, sms);
+    b2::ragged_worklist_kernel<<<1 + fill, 1024, 0, st>>>(
         cu_seqlens_q, cu_seqlens_kv, nullptr, B, max_seqlen_q, max_seqlen_kv, total_q, total_kv, causal, Hkv, G / hpi,
         hpi, G, header, items, reinterpret_cast<int*>(wsb + wl.sorted_off), reinterpret_cast<int*>(wsb + wl.rank_off),
-        max_tiles, 0);
+        max_tiles, 0, fill ? lse : nullptr, max_seqlen_q, Hq);
     if (int e = launch_status()) return e;
-    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
-        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
-        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
-        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
-        if (int e = launch_status()) return e;
-    }
     pp.mode = 1;
     pp.B = B;
     pp.Hq = Hq;
@@ -609,12 +613,6 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     const int qmax = wl.qmax;
     char* wsb = static_cast<char*>(workspace);
 
-    if (lse != nullptr && lse_base == ATTN_LSE_PADDED_BSH) {
-        const int64_t n = (int64_t)B * max_seqlen_q * Hq;
-        const int blocks = (int)((n + 255) / 256 < (int64_t)sms * 8 ? (n + 255) / 256 : (int64_t)sms * 8);
-        b2::lse_padded_fill_kernel<<<blocks, 256, 0, st>>>(cu_seqlens_q, B, max_seqlen_q, Hq, lse);
-        if (int e = launch_status()) return e;
-    }
     const int dev_lse_layout = (lse_base == ATTN_LSE_PADDED_BSH) ? 1 : (lse_base == ATTN_LSE_PACKED_TH) ? 2 : 3;
 
     // ---- sequences of 1..qmax queries (decode, multi-token decode): split-KV decode kernel
@@ -702,10 +700,13 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
     int* header = reinterpret_cast<int*>(wsb);
     int4* items = reinterpret_cast<int4*>(wsb + wl.rw.items_off);
-    b2::ragged_worklist_kernel<<<1, 1024, 0, st>>>(
+    // blocks 1.. also write the padded LSE rows past each length (the short rows'
+    // merge and the prefill kernel write the rows inside)
+    const int fill = lse_fill_blocks(lse, lse_base, B, max_seqlen_q, Hq, sms);
+    b2::ragged_worklist_kernel<<<1 + fill, 1024, 0, st>>>(
         cu_seqlens_q, nullptr, kv_lens, B, max_seqlen_q, max_kv_len, total_q, 0, causal, Hkv, G / hpi, hpi, G,
         header, items, reinterpret_cast<int*>(wsb + wl.rw.sorted_off), reinterpret_cast<int*>(wsb + wl.rw.rank_off),
-        max_tiles, qmax);
+        max_tiles, qmax, fill ? lse : nullptr, max_seqlen_q, Hq);
     if (int e = launch_status()) return e;
     // the work-list kernel also validates every sequence; with all of them short
     // (max_seqlen_q <= qmax) its list is empty and the prefill kernel has nothing to do
