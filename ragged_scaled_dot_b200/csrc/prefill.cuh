@@ -158,6 +158,30 @@ __device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const C
     }
 }
 
+// Mode 2 with two page boxes per tile (64-row boxes, the common page size): both
+// page ids are read before either box is issued, so their latencies overlap
+// (each TMA issue is ordered after the reads before it).  id = -1 past Lkv.
+__device__ __forceinline__ void paged_tile_ids2(const PrefillParams& p, const int32_t* table, int64_t table_stride,
+                                                int b, int t0, int Lkv, int (&id)[2]) {
+    const int t1 = t0 + p.box_rows;
+    id[0] = (t0 < Lkv) ? page_lookup(table, table_stride, b, t0, p.page_size) : -1;
+    id[1] = (t1 < Lkv) ? page_lookup(table, table_stride, b, t1, p.page_size) : -1;
+}
+__device__ __forceinline__ void paged_issue_ids2(const PrefillParams& p, const CUtensorMap* map, const int (&id)[2],
+                                                 uint32_t dst, uint32_t bar, int g, int t0, int Lkv,
+                                                 uint32_t box_bytes) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int t = t0 + i * p.box_rows;
+        int gg = p.n_groups;
+        if (t < Lkv) {
+            const int page = page_checked(id[i], p.num_pages);
+            if (page >= 0) gg = page_group(page, page_slot(t, p.page_size), p.groups_per_page);
+        }
+        tma_load_5d(dst + (uint32_t)i * box_bytes, map, bar, 0, 0, 0, gg, g);
+    }
+}
+
 // Mode 2: does the K/V tile from t0 end inside a page box that runs past Lkv
 // (rows past the sequence that can hold stale values, possibly NaN)?
 __device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int t0, int Lkv) {
@@ -279,7 +303,10 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                 tma_load_5d(sQ + s * TILE, &p.tm_q, b_qfull, 0, it.q_tok0, 0, it.h0 + s, it.batch);
             ++q_it;
             const int g = it.h0 / p.G;
+            // with one table for K and V, the V boxes of a tile reuse the K boxes' page ids
+            const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
             for (int j = 0; ok && j < it.n_kv; ++j) {
+                int ids[2] = {-1, -1};
                 for (int t = 0; t < 2; ++t) {
                     const int st = kv_it % NST;
                     if (!mbar_wait(empty_bar(st), ((kv_it / NST) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -287,8 +314,16 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
                     if constexpr (PAGED) {
                         const uint32_t box_bytes = (uint32_t)p.box_rows * (D / 64) * 128u;
-                        paged_issue_tile(p, map, t ? p.v_page_table : p.page_table, t ? p.v_pt_stride : p.pt_stride,
-                                         sKV + st * TILE, full_bar(st), it.b, g, j * 128, it.Lkv, box_bytes);
+                        if (p.box_rows == 64) {
+                            if (t == 0 || !shared_table)
+                                paged_tile_ids2(p, t ? p.v_page_table : p.page_table, t ? p.v_pt_stride : p.pt_stride,
+                                                it.b, j * 128, it.Lkv, ids);
+                            paged_issue_ids2(p, map, ids, sKV + st * TILE, full_bar(st), g, j * 128, it.Lkv, box_bytes);
+                        } else {
+                            paged_issue_tile(p, map, t ? p.v_page_table : p.page_table,
+                                             t ? p.v_pt_stride : p.pt_stride, sKV + st * TILE, full_bar(st), it.b, g,
+                                             j * 128, it.Lkv, box_bytes);
+                        }
                         if (t == 1 && paged_tile_has_tail(p, j * 128, it.Lkv)) {
                             // value rows past the sequence: zero them once the tile lands, then
                             // release the tile to the MMA thread through this stage's tail barrier
