@@ -305,6 +305,9 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
             const int g = it.h0 / p.G;
             // with one table for K and V, the V boxes of a tile reuse the K boxes' page ids
             const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
+            // page ids of the next tile, read while this thread waits for a free stage
+            int ids_next[2] = {-1, -1};
+            bool have_next = false;
             for (int j = 0; ok && j < it.n_kv; ++j) {
                 int ids[2] = {-1, -1};
                 for (int t = 0; t < 2; ++t) {
@@ -315,10 +318,19 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                     if constexpr (PAGED) {
                         const uint32_t box_bytes = (uint32_t)p.box_rows * (D / 64) * 128u;
                         if (p.box_rows == 64) {
-                            if (t == 0 || !shared_table)
+                            if (t == 0 && have_next) {
+                                ids[0] = ids_next[0];
+                                ids[1] = ids_next[1];
+                            } else if (t == 0 || !shared_table) {
                                 paged_tile_ids2(p, t ? p.v_page_table : p.page_table, t ? p.v_pt_stride : p.pt_stride,
                                                 it.b, j * 128, it.Lkv, ids);
+                            }
                             paged_issue_ids2(p, map, ids, sKV + st * TILE, full_bar(st), g, j * 128, it.Lkv, box_bytes);
+                            if (t == 1) {
+                                have_next = j + 1 < it.n_kv;
+                                if (have_next)
+                                    paged_tile_ids2(p, p.page_table, p.pt_stride, it.b, (j + 1) * 128, it.Lkv, ids_next);
+                            }
                         } else {
                             paged_issue_tile(p, map, t ? p.v_page_table : p.page_table,
                                              t ? p.v_pt_stride : p.pt_stride, sKV + st * TILE, full_bar(st), it.b, g,
