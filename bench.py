@@ -47,7 +47,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 #     batch like the K/V bytes)
 #   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.6837 / 0.6345 GB)
 #   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7045 / 0.6711 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0262, "paged_prefill": 1.0776,
+TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0262, "paged_prefill": 1.0760,
                  "dense_prefill": 1.0497}
 
 
