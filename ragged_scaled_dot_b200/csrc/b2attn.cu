@@ -615,13 +615,32 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
 
     const int dev_lse_layout = (lse_base == ATTN_LSE_PADDED_BSH) ? 1 : (lse_base == ATTN_LSE_PACKED_TH) ? 2 : 3;
 
-    // ---- sequences of 1..qmax queries (decode, multi-token decode): split-KV decode kernel
+    // every tensor map is encoded (and may fail) before the first launch, so a host-side
+    // error leaves nothing enqueued
+    PrefillParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    if (encode_tok_tiles(&pp.tm_q, q, D, Hq, total_q, 1, q_strides[0], q_strides[1],
+                         unit_dim_stride(q_strides[0] * total_q, 8)))
+        return ATTN_ERR_INVALID_ARG;
+    {
+        // (column in block, row in 8-row group, 64-column block, 8-row group of the pool, head)
+        const uint64_t dims[5] = {64, 8, (uint64_t)(D / 64), (uint64_t)(num_pages * gk), (uint64_t)Hkv};
+        const uint32_t box[5] = {64, 8, (uint32_t)(D / 64), (uint32_t)(R / 8), 1};
+        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, 8 * k_pool_strides[1] * 2, k_pool_strides[2] * 2};
+        const int64_t sv[4] = {v_pool_strides[1] * 2, 128, 8 * v_pool_strides[1] * 2, v_pool_strides[2] * 2};
+        if (encode_5d(&pp.tm_k, k_pool, dims, sk, box) || encode_5d(&pp.tm_v, v_pool, dims, sv, box))
+            return ATTN_ERR_INVALID_ARG;
+    }
+    DecodeParams dp;
+    std::memset(&dp, 0, sizeof(dp));
     if (qmax > 0) {
-        DecodeParams dp;
-        std::memset(&dp, 0, sizeof(dp));
         if (int e = encode_decode_pool_maps(dp, k_pool, v_pool, D, D, page_size, Hkv, num_pages, k_pool_strides,
                                             v_pool_strides))
             return e;
+    }
+
+    // ---- sequences of 1..qmax queries (decode, multi-token decode): split-KV decode kernel
+    if (qmax > 0) {
         dp.q = static_cast<const __nv_bfloat16*>(q);
         dp.q_bs = q_strides[0];
         dp.q_hs = q_strides[1];
@@ -680,21 +699,8 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         }
     }
 
-    // ---- the other sequences: tcgen05 prefill kernel over page boxes
-    PrefillParams pp;
-    std::memset(&pp, 0, sizeof(pp));
-    if (encode_tok_tiles(&pp.tm_q, q, D, Hq, total_q, 1, q_strides[0], q_strides[1],
-                         unit_dim_stride(q_strides[0] * total_q, 8)))
-        return ATTN_ERR_INVALID_ARG;
-    {
-        // (column in block, row in 8-row group, 64-column block, 8-row group of the pool, head)
-        const uint64_t dims[5] = {64, 8, (uint64_t)(D / 64), (uint64_t)(num_pages * gk), (uint64_t)Hkv};
-        const uint32_t box[5] = {64, 8, (uint32_t)(D / 64), (uint32_t)(R / 8), 1};
-        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, 8 * k_pool_strides[1] * 2, k_pool_strides[2] * 2};
-        const int64_t sv[4] = {v_pool_strides[1] * 2, 128, 8 * v_pool_strides[1] * 2, v_pool_strides[2] * 2};
-        if (encode_5d(&pp.tm_k, k_pool, dims, sk, box) || encode_5d(&pp.tm_v, v_pool, dims, sv, box))
-            return ATTN_ERR_INVALID_ARG;
-    }
+    // ---- the other sequences: tcgen05 prefill kernel over page boxes (tensor maps
+    // encoded above, before anything was enqueued)
     int hpi, n_pairs;
     pair_shape(Hq, Hkv, &hpi, &n_pairs);
     const int max_tiles = ragged_max_tiles(B, max_seqlen_q, total_q);
