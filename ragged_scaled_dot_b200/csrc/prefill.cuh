@@ -14,7 +14,12 @@
 // Warp roles (320 threads):
 //   warp 0      claims items, publishes them to the other roles through a
 //               small shared-memory ring, and issues the TMA loads: Q tiles of
-//               the item, then K(j), V(j) into a ring of NST stages.
+//               the item, then K(j), V(j) into a ring of NST stages.  Over a
+//               paged cache it also reads the page ids; with 64-row page boxes
+//               a tile's two ids are read together, the V boxes reuse the K
+//               boxes' ids, and the next tile's ids are read while it waits for
+//               a free stage (one thread doing these reads one by one could not
+//               keep up with the MMAs).
 //   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit
 //               (descriptor bases are precomputed: this thread shares its SM
 //               sub-partition with two busy softmax warps, so every instruction
