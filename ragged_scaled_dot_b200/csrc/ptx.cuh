@@ -115,8 +115,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // ---------------------------------------------------------------------------
 // Thread-block clusters: rank, the cluster-wide barrier, addresses in a peer
-// CTA's shared memory, arrivals on a peer's mbarrier, and bulk copies from this
-// CTA's shared memory into a peer's (completion counted on the peer's barrier).
+// CTA's shared memory, arrivals on a peer's mbarrier, and stores into a peer's
+// shared memory (completion counted on the peer's barrier).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
@@ -132,7 +132,7 @@ __device__ __forceinline__ uint32_t peer_smem(uint32_t local, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
     return r;
 }
-// Relaxed (no release ordering): for signals whose payload travels by bulk copy
+// Relaxed (no release ordering): for signals whose payload travels by st.async
 // (completed through the barrier's transaction count) or that only follow an
 // observed tensor-core completion.  A release at cluster scope here measured
 // 0.5-1.5 us per arrival on B200.
@@ -143,16 +143,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_peer_relaxed(uint32_t clus
     asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
                  "r"(bytes)
                  : "memory");
-}
-// bytes (multiple of 16) from this CTA's shared memory at src to dst in the
-// cluster window; both 16-byte aligned.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
-                                                  uint32_t cluster_bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src), "r"(bytes), "r"(cluster_bar)
-        : "memory");
 }
 
 // Asynchronous stores into a peer CTA's shared memory (cluster window address)
@@ -278,14 +268,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
           "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
