@@ -1,4 +1,4 @@
-"""The four measured workloads at full size, in the launch configuration the
+"""The measured workloads at full size, in the launch configuration the
 bench times (same seeds, same split counts), checked against the fp64 oracle on
 sampled rows: the first and last query row of every sequence, rows on both
 sides of every 128-row tile boundary of a few sequences, and random rows."""
@@ -153,3 +153,66 @@ def test_paged_prefill_full_size():
         assert_lse_close(lse[b, tok - int(cu_q[b]), hh], l_ref, f"paged prefill full b={b}")
         n_checked += len(rows)
     assert n_checked >= 512 + 16 * 2
+
+
+def test_mixed_batch_full_size():
+    """The mixed batch at full size, in the bench's launch configuration (its
+    suggested split count for the short rows, token-major LSE): every row of the
+    48 short sequences for every head, and on the 16 chunk sequences the first
+    and last rows, both sides of each 128-row tile boundary and of each page
+    boundary, plus 512 random rows, against the oracle over each sequence's keys
+    gathered from the pool."""
+    w = synth.WORKLOADS["mixed_batch"]
+    q, kp, vp, table, kl, cu_q, lq = synth.make_mixed_batch(w, DEV)
+    T, smax = int(cu_q[-1]), int(lq.max())
+    L = kl.astype(np.int64)
+    n_short = int(np.sum((lq >= 1) & (lq <= 4)))
+    num_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    S = rsd.attn_paged_suggest_splits(max(1, n_short), w.Hq, w.Hkv, w.Dqk, w.Dv, int(L.max()), w.page_size, num_sms)
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((T, w.Hq), float("nan"), dtype=torch.float32, device=DEV)
+    ws = torch.full((rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv, w.Dqk, S),), 0xFF,
+                    dtype=torch.uint8, device=DEV)
+    rsd.attn_fwd_paged_prefill(q, kp, vp, o, lse, torch.as_tensor(cu_q, device=DEV),
+                               torch.as_tensor(table, device=DEV), torch.as_tensor(kl, device=DEV),
+                               max_seqlen_q=smax, page_size=w.page_size, max_kv_len=int(L.max()),
+                               scale=w.scale, causal=True, workspace=ws, num_splits=S,
+                               lse_layout=rsd.ATTN_LSE_PACKED_TH)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    assert not torch.isnan(o).any() and not torch.isnan(lse).any()
+    rng = np.random.default_rng(5)
+    extra = {b: [] for b in range(w.B)}
+    chunks = [b for b in range(w.B) if lq[b] > 4]
+    for _ in range(512):
+        b = chunks[int(rng.integers(len(chunks)))]
+        extra[b].append(int(rng.integers(int(lq[b]))))
+    n_checked = 0
+    for b in range(w.B):
+        Lb, n = int(L[b]), int(lq[b])
+        if n == 0:
+            continue
+        if n <= 4:
+            rows = np.array([(0, h, i) for i in range(n) for h in range(w.Hq)], dtype=np.int32)
+        else:
+            idx = {0, n - 1}
+            for t in range(128, n, 128):
+                idx |= {t - 1, t}
+            first_pos = Lb - n
+            for pos in range((first_pos // w.page_size + 1) * w.page_size, Lb, w.page_size):
+                idx |= {pos - 1 - first_pos, pos - first_pos}
+            idx = sorted(i for i in idx | set(extra[b]) if 0 <= i < n)
+            rows = np.array([(0, int(rng.integers(w.Hq)), i) for i in idx], dtype=np.int32)
+        j = np.arange(Lb)
+        pages = torch.as_tensor(table[b, j // w.page_size].astype(np.int64), device=DEV)
+        slots = torch.as_tensor(j % w.page_size, device=DEV)
+        kc, vc = kp[pages, :, slots].contiguous(), vp[pages, :, slots].contiguous()
+        q_b = q[int(cu_q[b]):int(cu_q[b + 1])]
+        o_ref, l_ref = orc().attn_ragged_rows(bits(q_b), bits(kc), bits(vc), np.array([0, n]),
+                                              np.array([0, Lb]), w.Hq, w.Hkv, w.scale, True, rows)
+        tok = torch.as_tensor(rows[:, 2].astype(np.int64) + int(cu_q[b]), device=DEV)
+        hh = torch.as_tensor(rows[:, 1].astype(np.int64), device=DEV)
+        assert_o_close(o[tok, hh], o_ref, f"mixed batch full b={b}")
+        assert_lse_close(lse[tok, hh], l_ref, f"mixed batch full b={b}")
+        n_checked += len(rows)
+    assert n_checked >= 512 + 48 * w.Hq
