@@ -95,21 +95,41 @@ __device__ __forceinline__ uint32_t decode_chunk_bytes(const DecodeParams& p, in
     return (uint32_t)nboxes * (uint32_t)p.box_rows * 128u * (uint32_t)ncol_blocks * (uint32_t)tensors;
 }
 
-// Issues the TMA loads of that chunk for kv head g of sequence b: rows
-// [r, r + box_rows) of the chunk come from one page (lookup in `table`, the K
-// or the V page table).
-__device__ __forceinline__ void decode_issue_chunk(const DecodeParams& p, const CUtensorMap* map,
-                                                   const int32_t* table, int64_t table_stride,
-                                                   uint32_t dst, uint32_t bar, int b, int g, int t0,
-                                                   int hi, int ncol_blocks, uint32_t block_bytes) {
-    const int nkeys = min(64, hi - t0);
-    for (int r = 0; r < nkeys; r += p.box_rows) {
-        const int t = t0 + r;
-        // out of range: page -1, and TMA fills the box with zeros
-        const int page = page_checked(page_lookup(table, table_stride, b, t, p.page_size), p.num_pages);
-        const int slot = page_slot(t, p.page_size);
-        for (int cb = 0; cb < ncol_blocks; ++cb)
-            tma_load_4d(dst + cb * block_bytes + (uint32_t)r * 128u, map, bar, cb * 64, slot, g, page);
+// Issues the K and V TMA loads of the chunk from t0 for kv head g of sequence b:
+// rows [r, r + box_rows) come from one page (NB = 64 / box_rows boxes).  All
+// page ids of the chunk are read before any box is issued, so their latencies
+// overlap (each TMA issue is ordered after the reads before it; one thread
+// reading them box by box could not keep a small batch's few blocks streaming),
+// and with one page table for K and V the V boxes reuse the K boxes' ids.
+template <int NB>
+__device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t dst_k, uint32_t dst_v, uint32_t bar,
+                                                int b, int g, int t0, int hi, int ncol_blocks, uint32_t block_bytes) {
+    const int R = p.box_rows;
+    const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
+    int idk[NB], idv[NB];
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+        const int t = t0 + i * R;
+        idk[i] = (t < hi) ? page_lookup(p.page_table, p.pt_stride, b, t, p.page_size) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+        const int t = t0 + i * R;
+        idv[i] = shared_table ? idk[i] : ((t < hi) ? page_lookup(p.v_page_table, p.v_pt_stride, b, t, p.page_size) : -1);
+    }
+#pragma unroll
+    for (int i = 0; i < NB; ++i) {
+        const int t = t0 + i * R;
+        if (t < hi) {
+            // out of range: page -1, and TMA fills the box with zeros
+            const int pk = page_checked(idk[i], p.num_pages);
+            const int pv = shared_table ? pk : page_checked(idv[i], p.num_pages);
+            const int slot = page_slot(t, p.page_size);
+            for (int cb = 0; cb < ncol_blocks; ++cb) {
+                tma_load_4d(dst_k + cb * block_bytes + (uint32_t)(i * R) * 128u, &p.tm_k, bar, cb * 64, slot, g, pk);
+                tma_load_4d(dst_v + cb * block_bytes + (uint32_t)(i * R) * 128u, &p.tm_v, bar, cb * 64, slot, g, pv);
+            }
+        }
     }
 }
 
@@ -192,10 +212,12 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 const int t0 = lo + c * 64;
                 mbar_arrive_expect_tx(full_bar(st), decode_chunk_bytes(p, t0, hi, C::NCB, 2));
                 const uint32_t dst = sb + st * C::STAGE;
-                decode_issue_chunk(p, &p.tm_k, p.page_table, p.pt_stride, dst, full_bar(st), b, g, t0, hi, C::NCB,
-                                   C::BLK);
-                decode_issue_chunk(p, &p.tm_v, p.v_page_table, p.v_pt_stride, dst + C::CHUNK, full_bar(st), b, g,
-                                   t0, hi, C::NCB, C::BLK);
+                switch (64 / p.box_rows) {
+                    case 1: decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
+                    case 2: decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
+                    case 4: decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
+                    default: decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
+                }
             }
             // drain: every issued load lands before the block leaves
             for (int c = max(0, n_chunks - NST); c < n_chunks; ++c)
