@@ -279,8 +279,10 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
         const uint32_t sV = sK + C::CHUNK;
         const int t0 = lo + c * 64;
         const int nvalid = min(64, hi - t0);
+        bool zeroed = false;
         if (active) {
             if (kbase + KW > nvalid) {
+                zeroed = true;
                 // V rows past the split (or never loaded) must be finite: zero them.
                 uint8_t* vg = sgen + (sV - sb);
                 for (int i = lane; i < KW * C::NCB * 8; i += 32) {
@@ -293,9 +295,15 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 __syncwarp();
             }
             // S = Q K^T over this warp's keys (n-tiles of 8 keys)
-            float sacc[2 * RT][4];
+            // with RT <= 2, two accumulators per n-tile (even and odd k-steps), so each chain
+            // of dependent MMAs is half as long (RT = 4 has enough independent chains and
+            // no registers to spare)
+            constexpr bool kTwoChains = RT <= 2;
+            float sacc[2 * RT][4], sacc2[2 * RT][4];
 #pragma unroll
-            for (int nt = 0; nt < 2 * RT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            for (int nt = 0; nt < 2 * RT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.f;
             {
                 const int mat = lane >> 3, rr = lane & 7;
 #pragma unroll
@@ -307,9 +315,17 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                         const int dcol = (kk & 3) * 16 + ((mat & 1) << 3);
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4(sK + cb * C::BLK + sw128_offset(key, dcol), b0, b1, b2, b3);
-                        mma_bf16_16816(sacc[2 * kg], qa[kk], b0, b1);
-                        mma_bf16_16816(sacc[2 * kg + 1], qa[kk], b2, b3);
+                        float (&a0)[4] = (kTwoChains && (kk & 1)) ? sacc2[2 * kg] : sacc[2 * kg];
+                        float (&a1)[4] = (kTwoChains && (kk & 1)) ? sacc2[2 * kg + 1] : sacc[2 * kg + 1];
+                        mma_bf16_16816(a0, qa[kk], b0, b1);
+                        mma_bf16_16816(a1, qa[kk], b2, b3);
                     }
+                }
+                if constexpr (kTwoChains) {
+#pragma unroll
+                    for (int nt = 0; nt < 2 * RT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
                 }
             }
             // online softmax (log2 domain, scale folded in); keys outside a row's range masked
@@ -328,10 +344,15 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
             for (int hh = 0; hh < 2; ++hh) {
                 mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
                 mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+                // the reference maximum moves only when a score exceeds it by more than 8
+                // (P stays <= 2^8), so most chunks leave O and l as they are
                 const float mn = fmaxf(m[hh], mx[hh]);
-                alpha[hh] = (m[hh] == -INFINITY) ? 0.f : ex2(m[hh] - mn);
-                m[hh] = mn;
-                mref[hh] = (mn == -INFINITY) ? 0.f : mn;
+                alpha[hh] = 1.f;
+                if (mn > m[hh] + 8.f) {
+                    alpha[hh] = (m[hh] == -INFINITY) ? 0.f : ex2(m[hh] - mn);
+                    m[hh] = mn;
+                }
+                mref[hh] = (m[hh] == -INFINITY) ? 0.f : m[hh];
             }
             float psum[2] = {0.f, 0.f};
 #pragma unroll
@@ -344,12 +365,14 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 }
             l[0] = l[0] * alpha[0] + psum[0];
             l[1] = l[1] * alpha[1] + psum[1];
+            if (alpha[0] != 1.f || alpha[1] != 1.f) {
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                oacc[i][0] *= alpha[0];
-                oacc[i][1] *= alpha[0];
-                oacc[i][2] *= alpha[1];
-                oacc[i][3] *= alpha[1];
+                for (int i = 0; i < D / 8; ++i) {
+                    oacc[i][0] *= alpha[0];
+                    oacc[i][1] *= alpha[0];
+                    oacc[i][2] *= alpha[1];
+                    oacc[i][3] *= alpha[1];
+                }
             }
             // O += P V over this warp's keys, 16 keys per k-step
             const int mat = lane >> 3, rr = lane & 7;
@@ -372,7 +395,9 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 }
             }
         }
-        fence_proxy_async_smem();
+        // generic writes to the stage (the zeroed V rows) are ordered before the next TMA
+        // writes into it; reads need only the barrier
+        if (zeroed) fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(st));
     }
