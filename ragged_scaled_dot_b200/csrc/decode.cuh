@@ -103,19 +103,26 @@ __device__ __forceinline__ uint32_t decode_chunk_bytes(const DecodeParams& p, in
 // and with one page table for K and V the V boxes reuse the K boxes' ids.
 template <int NB>
 __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t dst_k, uint32_t dst_v, uint32_t bar,
-                                                int b, int g, int t0, int hi, int ncol_blocks, uint32_t block_bytes) {
+                                                int b, int g, int t0, int hi, int ncol_blocks, uint32_t block_bytes,
+                                                const volatile int* ids_k, const volatile int* ids_v, int p0, int nids) {
     const int R = p.box_rows;
     const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
     int idk[NB], idv[NB];
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
         const int t = t0 + i * R;
-        idk[i] = (t < hi) ? page_lookup(p.page_table, p.pt_stride, b, t, p.page_size) : -1;
+        const int w = t / p.page_size - p0;  // position in the window of shared-memory ids
+        idk[i] = (t >= hi) ? -1 : (w < nids ? ids_k[w] : page_lookup(p.page_table, p.pt_stride, b, t, p.page_size));
     }
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
         const int t = t0 + i * R;
-        idv[i] = shared_table ? idk[i] : ((t < hi) ? page_lookup(p.v_page_table, p.v_pt_stride, b, t, p.page_size) : -1);
+        const int w = t / p.page_size - p0;
+        idv[i] = shared_table ? idk[i]
+                              : ((t >= hi) ? -1
+                                           : (w < nids ? ids_v[w]
+                                                       : page_lookup(p.v_page_table, p.v_pt_stride, b, t,
+                                                                     p.page_size)));
     }
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
@@ -155,7 +162,11 @@ struct DecodeCfg {
     static constexpr int NST = 3;
     static constexpr uint32_t STAGE = 2 * CHUNK;        // K then V
     static constexpr uint32_t BAR_OFF = NST * STAGE;
-    static constexpr uint32_t SMEM = BAR_OFF + 128 + 1024;
+    // the block's page ids (K table, then V table when it has its own), read once at the
+    // start by every thread: the producer thread then finds them in shared memory
+    static constexpr int IDW = 1024;                  // page ids per table in the window
+    static constexpr uint32_t IDS_OFF = BAR_OFF + 128;
+    static constexpr uint32_t SMEM = IDS_OFF + 2 * IDW * 4 + 1024;
 };
 
 template <int D, int RT>
@@ -200,6 +211,20 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
         *abort_flag = 0;
         fence_barrier_init();
     }
+    // the page ids of keys [lo, hi) (up to IDW per table), read once by every thread
+    volatile int* ids_k = reinterpret_cast<volatile int*>(sgen + C::IDS_OFF);
+    volatile int* ids_v = ids_k + C::IDW;
+    const int p0 = lo / p.page_size;
+    const int nids = (hi > lo) ? min(C::IDW, (hi - 1) / p.page_size - p0 + 1) : 0;
+    {
+        const bool own_v = !(p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride);
+        const int32_t* rk = p.page_table + (int64_t)b * p.pt_stride + p0;
+        const int32_t* rv = p.v_page_table + (int64_t)b * p.v_pt_stride + p0;
+        for (int i = threadIdx.x; i < nids; i += blockDim.x) {
+            ids_k[i] = __ldg(rk + i);
+            if (own_v) ids_v[i] = __ldg(rv + i);
+        }
+    }
     __syncthreads();
 
     if (warp == 4) {
@@ -213,10 +238,22 @@ __global__ void __launch_bounds__(160) decode_gqa_kernel(const __grid_constant__
                 mbar_arrive_expect_tx(full_bar(st), decode_chunk_bytes(p, t0, hi, C::NCB, 2));
                 const uint32_t dst = sb + st * C::STAGE;
                 switch (64 / p.box_rows) {
-                    case 1: decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
-                    case 2: decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
-                    case 4: decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
-                    default: decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK); break;
+                    case 1:
+                        decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK, ids_k,
+                                           ids_v, p0, nids);
+                        break;
+                    case 2:
+                        decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK, ids_k,
+                                           ids_v, p0, nids);
+                        break;
+                    case 4:
+                        decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK, ids_k,
+                                           ids_v, p0, nids);
+                        break;
+                    default:
+                        decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK, ids_k,
+                                           ids_v, p0, nids);
+                        break;
                 }
             }
             // drain: every issued load lands before the block leaves
