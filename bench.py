@@ -339,7 +339,8 @@ def make_mixed(torch, rsd, synth, dev, seed_offset, num_sms, subset="all"):
     short = (lq >= 1) & (lq <= 4)
     kv_short = float(np.sum(L[short])) * w.Hkv * (w.Dqk + w.Dv) * 2
     qmax = min(4, 64 // (w.Hq // w.Hkv), smax)
-    launches = 1 + (1 + (2 if S > 1 else 0) if qmax > 0 else 0) + (1 if smax > qmax else 0)
+    # the work list; the short rows' decode (after its split schedule); the prefill kernel
+    launches = 1 + (1 + (1 if S > 1 else 0) if qmax > 0 else 0) + (1 if smax > qmax else 0)
     info = {"workload": w.notes, "subset": subset, "num_splits_short_rows": S, "query_tokens": T,
             "short_sequences": n_short, "chunk_sequences": int(np.sum(lq > 4)), "flop_per_step": flops,
             "kv_bytes_short_rows": kv_short, "traffic_basis_gb": kv_short / 1e9}
@@ -413,7 +414,9 @@ def make_paged(torch, rsd, synth, dev, seed_offset, name, num_sms, B=0):
             "flop_per_step": flops, "total_pages": int(kp.shape[0]),
             "bytes_per_unit": f"{w.Hkv * (w.Dqk if w.v_aliases_k else w.Dqk + Dv) * 2} B of K/V per cached token"}
     data = dict(q=q, kp=kp, vp=vp, table=table, L=L, w=w, S=S)
-    launches = 3 if S > 1 else 1  # with splits: the launch-order sort, the decode, the merge
+    # with splits: GQA the split schedule and the decode (which merges), MLA the launch-order
+    # sort, the decode and the merge
+    launches = (3 if w.Dqk == 576 else 2) if S > 1 else 1
     return Part(name, "GB/s", nbytes / 1e9, launches, step, e2e_setup, info), data
 
 

@@ -203,8 +203,8 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  * its kv_lens[b] cached keys ("cuDNN Frontend v1.31.0 Release Notes", "SDPA:
  * paged KV, split-KV, and engine selection").
  *   q: [B, Hq, Dqk] with (batch, head) element strides q_strides[2].
- *   o: [B, Hq, Dv]  with (batch, head) element strides o_strides[2]; with
- *   num_splits > 1 the rows must be batch-major (o_strides[0] == Hq *
+ *   o: [B, Hq, Dv]  with (batch, head) element strides o_strides[2]; for MLA
+ *   with num_splits > 1 the rows must be batch-major (o_strides[0] == Hq *
  *   o_strides[1]), else ATTN_ERR_UNSUPPORTED before anything is enqueued.
  *   lse (nullable): fp32 [B, Hq] contiguous.
  *   k_pool / v_pool: pools of num_pages fixed-size pages; element
@@ -222,13 +222,19 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  *   Each page-table row holds at least ceil(max_kv_len / page_size) entries.
  *   kv_lens: DEVICE int32 [B], each in [0, max_kv_len]; page ids must lie in
  *   [0, num_pages).  Violations set ATTN_ERR_DEVICE_INPUT on the device.
- * Split-KV: each sequence's pages are cut into num_splits ranges of
- * ceil(n_pages / num_splits) consecutive pages; num_splits > 1 writes fp32
- * partial O and LSE into the workspace and merges them as attn_split_merge
- * does, and the blocks take the sequences longest first (a device-side sort
- * of kv_lens into the workspace; it changes which block computes a split,
- * never the result).  workspace: >= attn_fwd_paged_workspace_size(...) bytes,
- * 256-byte aligned (may be NULL when num_splits == 1).
+ * Split-KV (num_splits > 1), GQA: the keys of each (sequence, KV head) are
+ * cut into 64-key units, and its n units into min(num_splits, n) pieces of
+ * n / pieces units (to within one), one block per piece, the sequences
+ * longest first (a device-side schedule in the workspace).  A piece that is
+ * the whole sequence writes O directly; the others write fp32 partial O and
+ * LSE, merged by LSE (as attn_split_merge does) inside the same launch by the
+ * last block to finish each group of up to 8 of a sequence's partials.  MLA:
+ * each sequence's pages are cut into num_splits ranges of ceil(n_pages /
+ * num_splits) pages, the clusters take the sequences longest first and a
+ * second launch merges the partials.  The schedule changes which block
+ * computes a piece, never the result.  workspace: >=
+ * attn_fwd_paged_workspace_size(...) bytes, 256-byte aligned (may be NULL
+ * when num_splits == 1).
  */
 int attn_fwd_paged(const void *q, const void *k_pool, const void *v_pool, void *o,
                    float *lse, const int32_t *page_table, int64_t page_table_stride,
@@ -281,8 +287,8 @@ int attn_fwd_paged_kv_tables(const void *q, const void *k_pool, const void *v_po
  * tensor-core prefill kernel in 128-row query tiles.  The split is decided on
  * the device from cu_seqlens_q (no host read); results do not depend on it.
  * num_splits (>= 1) splits the keys of each short sequence as attn_fwd_paged
- * does (fp32 partials in the workspace, merged by LSE); it does not affect
- * the other sequences.  attn_paged_suggest_splits gives a count.
+ * does for GQA (pieces of 64-key units, fp32 partials in the workspace merged
+ * by LSE in the same launch); it does not affect the other sequences.  attn_paged_suggest_splits gives a count.
  * Supported: D = Dqk = Dv in {64, 128}, Hq % Hkv == 0, page_size dividing 128
  * (at least 8) or a multiple of 128, and pools whose page stride is a whole
  * number of 8-row groups (page stride % (8 * row stride) == 0, the same for K
@@ -320,16 +326,17 @@ int attn_fwd_paged_prefill_kv_tables(const void *q, const void *k_pool, const vo
                                      void *stream);
 
 /* Workspace bytes attn_fwd_paged_prefill needs: the prefill work list (as for
- * attn_fwd_ragged) and, with num_splits > 1, the fp32 partials of the short
- * rows (B * qmax * Hq rows of D floats per split) and their launch order
- * (caller workspace as in "cuDNN Frontend v1.31.0 Release Notes",
- * "Compatibility and numerical behavior").  Host-only arithmetic; 0 for
- * invalid arguments. */
+ * attn_fwd_ragged) and, with num_splits > 1, the short rows' split schedule,
+ * merge counters and fp32 partials (num_splits * B * Hkv pieces of
+ * Hq / Hkv * qmax rows of D floats) (caller workspace as in "cuDNN Frontend
+ * v1.31.0 Release Notes", "Compatibility and numerical behavior").  Host-only
+ * arithmetic; 0 for invalid arguments. */
 size_t attn_fwd_paged_prefill_workspace_size(int B, int max_seqlen_q, int64_t total_q, int Hq, int Hkv,
                                              int D, int num_splits);
 
-/* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1): the fp32
- * split partials and the launch order live in caller-owned scratch ("cuDNN
+/* Workspace bytes attn_fwd_paged needs (0 when num_splits == 1): the split
+ * schedule, the merge counters and the fp32 partials (MLA: the partials and the
+ * launch order) live in caller-owned scratch ("cuDNN
  * Frontend v1.31.0 Release Notes", "Compatibility and numerical behavior":
  * split-attention calls require caller workspace, sized by a query). */
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits);

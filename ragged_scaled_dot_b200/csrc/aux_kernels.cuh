@@ -266,59 +266,16 @@ __global__ void __launch_bounds__(256) dense_worklist_kernel(int B, int Sq, int 
     }
 }
 
-// Launch order of a paged decode: sequence indices by cached length, longest
-// first, so the blocks of the longest splits start first and the short ones
-// fill in at the end (list scheduling in longest-processing-time order; the
-// splits of one sequence are equal to within a page).  Counting sort over
-// 4096 buckets of key = min(4095, L >> shift), the host choosing shift so that
-// max_kv_len >> shift < 4096.  Ties land in any order: the order only decides
-// which block runs a (sequence, split), never what it computes.  One block of
-// 1024 threads.
-__global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restrict__ kv_lens, int B, int max_kv_len,
-                                                         int shift, int32_t* __restrict__ order,
-                                                         const int32_t* __restrict__ cu_q, int qmax) {
-    __shared__ int hist[kSortBuckets];
-    __shared__ int warp_sums[32];
-    const int tid = threadIdx.x;
-    // bucket 0 holds the longest sequences; with ragged queries (cu_q), the
-    // sequences the decode kernel skips (not 1..qmax queries) count as empty
-    auto bucket = [&](int b) {
-        int L = max(0, min(__ldg(kv_lens + b), max_kv_len));
-        if (cu_q != nullptr) {
-            const int lq = __ldg(cu_q + b + 1) - __ldg(cu_q + b);
-            if (lq < 1 || lq > qmax) L = 0;
-        }
-        return kSortBuckets - 1 - min(kSortBuckets - 1, L >> shift);
-    };
-    for (int i = tid; i < kSortBuckets; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
-    for (int b = tid; b < B; b += blockDim.x) atomicAdd(&hist[bucket(b)], 1);
-    __syncthreads();
-    // exclusive scan of the buckets: thread t owns buckets [t*per, (t+1)*per)
+// In-place exclusive prefix of the kSortBuckets counts in hist, by a block of
+// 1024 threads (thread t owns buckets [t*per, (t+1)*per)); ends synchronised.
+__device__ __forceinline__ void bucket_exclusive_scan(int* hist, int* warp_sums) {
     constexpr int per = kSortBuckets / 1024;
+    const int tid = threadIdx.x;
     int local = 0;
 #pragma unroll
     for (int i = 0; i < per; ++i) local += hist[tid * per + i];
-    int incl = local;
-    const int lane = tid & 31, wid = tid >> 5;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-    }
-    if (lane == 31) warp_sums[wid] = incl;
-    __syncthreads();
-    if (wid == 0) {
-        int w = warp_sums[lane];
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += v;
-        }
-        warp_sums[lane] = w;  // inclusive prefix over warps
-    }
-    __syncthreads();
-    int run = incl - local + (wid > 0 ? warp_sums[wid - 1] : 0);
+    int total;
+    int run = block_exclusive_scan(local, warp_sums, &total);
 #pragma unroll
     for (int i = 0; i < per; ++i) {
         const int h = hist[tid * per + i];
@@ -326,6 +283,31 @@ __global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restri
         run += h;
     }
     __syncthreads();
+}
+
+// Launch order of a split MLA decode: sequence indices by cached length, longest
+// first, so the clusters of the longest splits start first and the short ones
+// fill in at the end (list scheduling in longest-processing-time order; the
+// splits of one sequence are equal to within a page).  Counting sort over
+// 4096 buckets of key = min(4095, L >> shift), the host choosing shift so that
+// max_kv_len >> shift < 4096.  Ties land in any order: the order only decides
+// which block runs a (sequence, split), never what it computes.  One block of
+// 1024 threads.
+__global__ void __launch_bounds__(1024) seq_order_kernel(const int32_t* __restrict__ kv_lens, int B, int max_kv_len,
+                                                         int shift, int32_t* __restrict__ order) {
+    __shared__ int hist[kSortBuckets];
+    __shared__ int warp_sums[32];
+    const int tid = threadIdx.x;
+    // bucket 0 holds the longest sequences
+    auto bucket = [&](int b) {
+        const int L = max(0, min(__ldg(kv_lens + b), max_kv_len));
+        return kSortBuckets - 1 - min(kSortBuckets - 1, L >> shift);
+    };
+    for (int i = tid; i < kSortBuckets; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int b = tid; b < B; b += blockDim.x) atomicAdd(&hist[bucket(b)], 1);
+    __syncthreads();
+    bucket_exclusive_scan(hist, warp_sums);
     for (int b = tid; b < B; b += blockDim.x) order[atomicAdd(&hist[bucket(b)], 1)] = b;
 }
 

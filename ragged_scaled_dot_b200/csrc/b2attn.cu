@@ -212,8 +212,55 @@ int noalloc_scratch(void** out) {
     return ATTN_OK;
 }
 
-// Launches the GQA decode kernel with RT 16-row m-tiles (1, 2 or 4) over grid
-// (num_splits, Hkv, B).
+// Split workspace of the GQA decode, from byte `base`: per-sequence {units, L,
+// q0, Lq} [B], the longest-first order [B], every block's piece [n_slots],
+// arrival counters [kMergeLevels][n_slots], partial O fp32 [n_slots][rps][Dv]
+// and base-2 LSE [n_slots][rps], each 256-byte aligned; n_slots = num_splits *
+// pairs, the blocks of the launch.
+struct SplitWs {
+    int64_t seq_off, order_off, segs_off, ctr_off, part_off, lse_off, total;
+};
+SplitWs split_ws_layout(int64_t base, int B, int64_t pairs, int64_t rps, int Dv, int num_splits) {
+    const int64_t slots = (int64_t)num_splits * pairs;
+    SplitWs w;
+    w.seq_off = base;
+    w.order_off = round_up(w.seq_off + (int64_t)B * 16, 256);
+    w.segs_off = round_up(w.order_off + (int64_t)B * 4, 256);
+    w.ctr_off = round_up(w.segs_off + slots * (int64_t)sizeof(b2::DecodeSeg), 256);
+    w.part_off = round_up(w.ctr_off + (int64_t)b2::kMergeLevels * slots * 4, 256);
+    w.lse_off = round_up(w.part_off + slots * rps * Dv * 4, 256);
+    w.total = round_up(w.lse_off + slots * rps * 4, 256);
+    return w;
+}
+
+// Blocks of a split GQA decode launch (num_splits per pair), or 0 when the grid
+// or the schedule's 32-bit arithmetic would overflow (the call is then
+// unsupported).
+int64_t split_blocks(int64_t pairs, int max_kv_len, int num_splits) {
+    const int64_t n = (int64_t)num_splits * pairs;
+    if (n >= ((int64_t)1 << 30) || pairs * ((int64_t)max_kv_len / 64 + 2) >= ((int64_t)1 << 30)) return 0;
+    return n;
+}
+
+// Points the decode parameters at a split workspace and enqueues its schedule.
+int launch_decode_schedule(DecodeParams& dp, char* wsb, const SplitWs& w, int64_t n_blocks, int max_kv_len,
+                           cudaStream_t st) {
+    dp.segs = reinterpret_cast<const b2::DecodeSeg*>(wsb + w.segs_off);
+    dp.ctr = reinterpret_cast<int*>(wsb + w.ctr_off);
+    dp.n_slots = (int)n_blocks;
+    dp.o_part = reinterpret_cast<float*>(wsb + w.part_off);
+    dp.lse_part = reinterpret_cast<float*>(wsb + w.lse_off);
+    // sort keys: units >> shift below the bucket count
+    int shift = 0;
+    while (((max_kv_len / 64 + 1) >> shift) >= b2::kSortBuckets) ++shift;
+    b2::decode_schedule_kernel<<<1, 1024, 0, st>>>(dp, shift, reinterpret_cast<int4*>(wsb + w.seq_off),
+                                                  reinterpret_cast<int32_t*>(wsb + w.order_off),
+                                                  reinterpret_cast<b2::DecodeSeg*>(wsb + w.segs_off), dp.ctr);
+    return launch_status();
+}
+
+// Launches the GQA decode kernel with RT 16-row m-tiles (1, 2 or 4): grid
+// (1, Hkv, B) without splits, one block per scheduled piece with them.
 int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, cudaStream_t st) {
     if (D == 128) {
         if (RT == 1) b2::decode_gqa_kernel<128, 1><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
@@ -514,23 +561,22 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void) { return kNoAllocScratchBytes; 
 
 namespace {
 // Paged-prefill workspace: the ragged work list, then (routed short rows with
-// splits) partial O fp32 [S][B*qmax*Hq][D], partial LSE [S][B*qmax*Hq] and the
-// decode launch order [B], each 256-byte aligned.
+// splits) the split workspace of their decode kernel.
 struct PagedPrefillWs {
     RaggedWs rw;
     int qmax;
-    int64_t part_off, lse_off, order_off, total;
+    SplitWs sw;
+    int64_t total;
 };
 PagedPrefillWs paged_prefill_ws_layout(int B, int max_sq, int64_t total_q, int Hq, int Hkv, int D, int num_splits) {
     PagedPrefillWs w;
     w.rw = ragged_ws_layout(B, max_sq, total_q, Hq, Hkv);
     w.qmax = routed_qmax(Hq / Hkv, max_sq);
-    w.part_off = w.lse_off = w.order_off = w.total = w.rw.total;
+    w.sw = SplitWs{};
+    w.total = w.rw.total;
     if (w.qmax > 0 && num_splits > 1) {
-        const int64_t R = (int64_t)B * w.qmax * Hq;
-        w.lse_off = w.part_off + round_up(R * num_splits * D * 4, 256);
-        w.order_off = w.lse_off + round_up(R * num_splits * 4, 256);
-        w.total = w.order_off + round_up((int64_t)B * 4, 256);
+        w.sw = split_ws_layout(w.rw.total, B, (int64_t)B * Hkv, (int64_t)(Hq / Hkv) * w.qmax, D, num_splits);
+        w.total = w.sw.total;
     }
     return w;
 }
@@ -633,10 +679,20 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     }
     DecodeParams dp;
     std::memset(&dp, 0, sizeof(dp));
+    // short rows: G * qmax query rows in RT m16 tiles; with splits, one block per piece
+    int RT = 1;
+    int64_t n_cta = 0;
+    const int64_t dec_pairs = (int64_t)B * Hkv;
     if (qmax > 0) {
         if (int e = encode_decode_pool_maps(dp, k_pool, v_pool, D, D, page_size, Hkv, num_pages, k_pool_strides,
                                             v_pool_strides))
             return e;
+        RT = (G * qmax + 15) / 16;
+        if (RT == 3) RT = 4;
+        if (num_splits > 1) {
+            n_cta = split_blocks(dec_pairs, max_kv_len, num_splits);
+            if (n_cta == 0) return ATTN_ERR_UNSUPPORTED;
+        }
     }
 
     // ---- sequences of 1..qmax queries (decode, multi-token decode): split-KV decode kernel
@@ -671,31 +727,10 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         dp.lse_hs = total_q;
         dp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
         if (num_splits > 1) {
-            dp.o_part = reinterpret_cast<float*>(wsb + wl.part_off);
-            dp.lse_part = reinterpret_cast<float*>(wsb + wl.lse_off);
-            int32_t* order = reinterpret_cast<int32_t*>(wsb + wl.order_off);
-            int shift = 0;
-            while ((max_kv_len >> shift) >= 4096) ++shift;
-            b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order, cu_seqlens_q, qmax);
-            if (int e = launch_status()) return e;
-            dp.order = order;
-        }
-        int RT = (G * qmax + 15) / 16;
-        if (RT == 3) RT = 4;
-        if (int e = launch_decode_gqa(dp, D, RT, dim3(num_splits, Hkv, B), st)) return e;
-        if (num_splits > 1) {
-            const int64_t rows = (int64_t)B * qmax * Hq;
-            const unsigned blocks = (unsigned)((rows + 7) / 8);
-            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
-            if (D == 128)
-                b2::split_merge_thd_kernel<128><<<blocks, 256, 0, st>>>(
-                    dp.o_part, dp.lse_part, num_splits, cu_seqlens_q, B, qmax, Hq, total_q, ob, o_strides[0],
-                    o_strides[1], lse, dev_lse_layout, max_seqlen_q, total_q, dp.lse_log2);
-            else
-                b2::split_merge_thd_kernel<64><<<blocks, 256, 0, st>>>(
-                    dp.o_part, dp.lse_part, num_splits, cu_seqlens_q, B, qmax, Hq, total_q, ob, o_strides[0],
-                    o_strides[1], lse, dev_lse_layout, max_seqlen_q, total_q, dp.lse_log2);
-            if (int e = launch_status()) return e;
+            if (int e = launch_decode_schedule(dp, wsb, wl.sw, n_cta, max_kv_len, st)) return e;
+            if (int e = launch_decode_gqa(dp, D, RT, dim3((unsigned)n_cta, 1, 1), st)) return e;
+        } else {
+            if (int e = launch_decode_gqa(dp, D, RT, dim3(1, Hkv, B), st)) return e;
         }
     }
 
@@ -757,9 +792,13 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
 size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits) {
     if (B <= 0 || Hq <= 0 || Dv <= 0 || num_splits <= 1) return 0;
     const int64_t R = (int64_t)B * Hq;
-    // partial O, partial LSE, launch order of the sequences
-    return (size_t)(round_up(R * num_splits * Dv * 4, 256) + round_up(R * num_splits * 4, 256) +
-                    round_up((int64_t)B * 4, 256));
+    if (Dv == 512) {
+        // MLA: partial O, partial LSE, launch order of the sequences
+        return (size_t)(round_up(R * num_splits * Dv * 4, 256) + round_up(R * num_splits * 4, 256) +
+                        round_up((int64_t)B * 4, 256));
+    }
+    // GQA: sized with B * Hq pairs of one row, it covers every Hkv (pairs * G rows = B * Hq)
+    return (size_t)split_ws_layout(0, B, R, 1, Dv, num_splits).total;
 }
 
 int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len, int page_size,
@@ -864,8 +903,8 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     for (int i = 0; i < 3; ++i)
         if (!stride_ok(k_pool_strides[i]) || !stride_ok(v_pool_strides[i])) return ATTN_ERR_INVALID_ARG;
     if (num_splits > 1) {
-        // the merge writes O row r = b*Hq + h at o + r*o_strides[1]: batch-major rows
-        if (o_strides[0] != (int64_t)Hq * o_strides[1]) return ATTN_ERR_UNSUPPORTED;
+        // the MLA merge writes O row r = b*Hq + h at o + r*o_strides[1]: batch-major rows
+        if (mla && o_strides[0] != (int64_t)Hq * o_strides[1]) return ATTN_ERR_UNSUPPORTED;
         const size_t need = attn_fwd_paged_workspace_size(B, Hq, Dv, num_splits);
         if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_ERR_WORKSPACE;
@@ -873,6 +912,15 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     int dev, sms;
     if (int e = setup_device(&dev, &sms)) return e;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // MLA: one cluster of two CTAs (score CTA, value CTA) per (b, split, group of 128 heads)
+    const int64_t mla_units = (int64_t)B * num_splits * ((Hq + 127) / 128);
+    if (mla && 2 * mla_units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+    // GQA with splits: one block per scheduled piece
+    int64_t n_cta = 0;
+    if (!mla && num_splits > 1) {
+        n_cta = split_blocks((int64_t)B * Hkv, max_kv_len, num_splits);
+        if (n_cta == 0) return ATTN_ERR_UNSUPPORTED;
+    }
 
     DecodeParams dp;
     std::memset(&dp, 0, sizeof(dp));
@@ -917,26 +965,23 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     dp.o_hs = o_strides[1];
     dp.lse = lse;
     const int64_t R = (int64_t)B * Hq;
-    if (num_splits > 1) {
-        char* wsb = static_cast<char*>(workspace);
-        dp.o_part = reinterpret_cast<float*>(wsb);
-        dp.lse_part = reinterpret_cast<float*>(wsb + round_up(R * num_splits * Dv * 4, 256));
-        // sequences longest first: the blocks of the longest splits start first
-        int32_t* order = reinterpret_cast<int32_t*>(wsb + round_up(R * num_splits * Dv * 4, 256) +
-                                                    round_up(R * num_splits * 4, 256));
-        int shift = 0;
-        while ((max_kv_len >> shift) >= 4096) ++shift;
-        b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order, nullptr, 1);
-        if (int e = launch_status()) return e;
-        dp.order = order;
-    }
+    char* wsb = static_cast<char*>(workspace);
     if (mla) {
-        // one cluster of two CTAs (score CTA, value CTA) per (b, split, group of 128 heads)
-        const int64_t units = (int64_t)B * num_splits * ((Hq + 127) / 128);
-        if (2 * units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
+        if (num_splits > 1) {
+            dp.o_part = reinterpret_cast<float*>(wsb);
+            dp.lse_part = reinterpret_cast<float*>(wsb + round_up(R * num_splits * Dv * 4, 256));
+            // sequences longest first: the clusters of the longest splits start first
+            int32_t* order = reinterpret_cast<int32_t*>(wsb + round_up(R * num_splits * Dv * 4, 256) +
+                                                        round_up(R * num_splits * 4, 256));
+            int shift = 0;
+            while ((max_kv_len >> shift) >= 4096) ++shift;
+            b2::seq_order_kernel<<<1, 1024, 0, st>>>(kv_lens, B, max_kv_len, shift, order);
+            if (int e = launch_status()) return e;
+            dp.order = order;
+        }
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3((unsigned)(2 * units), 1, 1);
+        cfg.gridDim = dim3((unsigned)(2 * mla_units), 1, 1);
         cfg.blockDim = dim3(b2::MlaTcCfg::THREADS, 1, 1);
         cfg.dynamicSmemBytes = b2::MlaTcCfg::SMEM;
         cfg.stream = st;
@@ -948,14 +993,18 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         if (cudaLaunchKernelEx(&cfg, b2::decode_mla_tc_kernel, dp) != cudaSuccess) return ATTN_ERR_LAUNCH;
-    } else {
-        // the G <= 16 query heads of a KV head fill one m16 tile
-        if (int e = launch_decode_gqa(dp, Dqk, 1, dim3(num_splits, Hkv, B), st)) return e;
+        if (int e = launch_status()) return e;
+        if (num_splits > 1)
+            return attn_split_merge(dp.o_part, dp.lse_part, num_splits, R, Dv, o, o_strides[1], lse, stream);
+        return ATTN_OK;
     }
-    if (int e = launch_status()) return e;
-    if (num_splits > 1)
-        return attn_split_merge(dp.o_part, dp.lse_part, num_splits, R, Dv, o, o_strides[1], lse, stream);
-    return ATTN_OK;
+    // GQA: the G <= 16 query heads of a KV head fill one m16 tile
+    if (num_splits > 1) {
+        const SplitWs sw = split_ws_layout(0, B, R, 1, Dv, num_splits);
+        if (int e = launch_decode_schedule(dp, wsb, sw, n_cta, max_kv_len, st)) return e;
+        return launch_decode_gqa(dp, Dqk, 1, dim3((unsigned)n_cta, 1, 1), st);
+    }
+    return launch_decode_gqa(dp, Dqk, 1, dim3(1, Hkv, B), st);
 }
 
 // ------------------------------------------------------------------ merge

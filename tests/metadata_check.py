@@ -18,6 +18,16 @@ head h0 of the pair, KV tiles the item visits)):
     group (batch, kv head, query tile longest first, head pair);
   * header[0] = item count; after the prefill ran, header[1] = item count +
     number of persistent CTAs (each CTA makes one claim past the end).
+
+Split decode (GQA, num_splits = S > 1):
+  * sequence b owns n_b = max(1, ceil(L_b / 64)) 64-key units when the decode
+    kernel takes its rows (always without cu_q; 1 <= Lq <= qmax with it), else 0;
+  * the order lists the sequences longest first by key min(4095, n_b >> shift),
+    shift the smallest with (max_kv_len // 64 + 1) >> shift < 4096, ties in any order;
+  * in that order each of a sequence's Hkv pairs p = b * Hkv + g takes k = min(S, n_b)
+    consecutive blocks slot0 .. slot0 + k - 1; block slot0 + s runs units
+    [s n_b // k, (s+1) n_b // k): record (p, j0, j1, slot0, k, L, q0, Lq); blocks past
+    the last piece have p = -1.
 """
 from __future__ import annotations
 
@@ -152,3 +162,61 @@ def page_coords(table, b_idx, t_idx, page_size, num_pages, groups_per_page):
         else:
             out.append((page, row, page * groups_per_page + row // 8))
     return np.array(out, dtype=np.int64).reshape(-1, 3)
+
+
+def decode_units(kv_lens, max_kv_len, cu_q=None, qmax=1):
+    """Per sequence (units, L, q0, Lq) by the rule above."""
+    out = []
+    for b in range(len(kv_lens)):
+        L = max(0, min(int(kv_lens[b]), max_kv_len))
+        q0, lq, mine = b, 1, True
+        if cu_q is not None:
+            a0, a1 = int(cu_q[b]), int(cu_q[b + 1])
+            q0, lq = a0, a1 - a0
+            mine = 1 <= lq <= qmax
+        out.append((max(1, -(-L // 64)) if mine else 0, L, q0, lq))
+    return out
+
+
+def decode_sort_shift(max_kv_len):
+    shift = 0
+    while ((max_kv_len // 64 + 1) >> shift) >= 4096:
+        shift += 1
+    return shift
+
+
+def decode_pieces(seq, order, Hkv, S):
+    """Expected piece records, one row per block, in the given sequence order."""
+    rows = []
+    for b in order:
+        n, L, q0, lq = seq[b]
+        k = min(S, n)
+        for g in range(Hkv):
+            slot0 = len(rows)
+            for s_ in range(k):
+                rows.append((b * Hkv + g, s_ * n // k, (s_ + 1) * n // k, slot0, k, L, q0, lq))
+    return rows
+
+
+def check_decode_pieces(order, seg_rows, kv_lens, Hkv, S, max_kv_len, cu_q=None, qmax=1):
+    """Device schedule (order [B], one record per block [S * B * Hkv, 8]) against the
+    rule: the order is a permutation, longest first by bucket; the records are the ones
+    the rule gives for that order, bit for bit; every unit of every pair is in one block."""
+    seq = decode_units(kv_lens, max_kv_len, cu_q, qmax)
+    order = [int(x) for x in order]
+    assert sorted(order) == list(range(len(seq))), "order is not a permutation"
+    shift = decode_sort_shift(max_kv_len)
+    keys = [min(SORT_CAP, seq[b][0] >> shift) for b in order]
+    assert all(a >= c for a, c in zip(keys, keys[1:])), "order is not longest first"
+    want = decode_pieces(seq, order, Hkv, S)
+    rows = np.asarray(seg_rows, dtype=np.int64).reshape(-1, 8)
+    assert len(rows) == S * len(seq) * Hkv, "one record per block of the launch"
+    for c, w in enumerate(want):
+        assert tuple(int(x) for x in rows[c]) == w, f"block {c}: {tuple(rows[c])} != {w}"
+    assert np.all(rows[len(want):, 0] == -1), "blocks past the last piece must be empty"
+    covered = set()
+    for p_, j0, j1, *_ in want:
+        for u in range(j0, j1):
+            assert (p_, u) not in covered, "unit in two blocks"
+            covered.add((p_, u))
+    assert len(covered) == Hkv * sum(s[0] for s in seq), "a unit is in no block"

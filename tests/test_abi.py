@@ -166,10 +166,15 @@ def test_paged_rejects_bad_args_on_host(lib):
                  None)
 
     assert call() == rsd.ATTN_ERR_WORKSPACE              # 3 splits need a workspace
-    # split outputs go through the merge, which needs batch-major O rows: refused on the
-    # host, before the workspace is even looked at
+    # split MLA outputs go through the merge kernel, which needs batch-major O rows: refused
+    # on the host, before the workspace is even looked at; the GQA blocks write rows by
+    # their (batch, head) strides, so there only the missing workspace is reported
+    kp_mla = L3(64 * 576, 576, 64 * 576)
+    assert f(fake, fake, fake, fake, None, fake, 64, fake, 4, 128, 1, 576, 512, 64, 100, 4096,
+             L2(128 * 576, 576), L2(128 * 512 + 8, 512), kp_mla, kp_mla, 0.04, 3, None, 0,
+             None) == rsd.ATTN_ERR_UNSUPPORTED
     assert f(fake, fake, fake, fake, None, fake, 64, fake, 4, 64, 8, 128, 128, 64, 100, 4096,
-             q2, L2(64 * 128 + 8, 128), kp, kp, 0.088, 3, None, 0, None) == rsd.ATTN_ERR_UNSUPPORTED
+             q2, L2(64 * 128 + 8, 128), kp, kp, 0.088, 3, None, 0, None) == rsd.ATTN_ERR_WORKSPACE
     assert call(Dqk=96, Dv=96) == rsd.ATTN_ERR_UNSUPPORTED
     assert call(ps=48) == rsd.ATTN_ERR_UNSUPPORTED        # neither divides nor is divided by 64
     assert call(Hkv=7) == rsd.ATTN_ERR_INVALID_ARG        # 64 % 7 != 0

@@ -297,8 +297,9 @@ def test_mla_decode_independent_kv_tables(splits):
 @pytest.mark.parametrize("mla", [False, True])
 def test_decode_batch_permutation_bitwise(mla):
     """With splits the blocks take the sequences longest first (a device-side
-    sort of kv_lens): permuting the batch permutes the outputs bit for bit, so
-    every split lands on its own sequence whatever block runs it."""
+    sort): permuting the batch permutes the outputs bit for bit, so every split
+    lands on its own sequence whatever block runs it (GQA: a pair's pieces and
+    their merge depend on its own length only)."""
     lens = [3000, 10, 700, 700, 1, 2049, 64]
     if mla:
         q, k, v, table, kl = _paged_inputs(lens, 128, 1, 576, 64, seed=79, Dv=512)
@@ -312,3 +313,37 @@ def test_decode_batch_permutation_bitwise(mla):
                        o_dv=Dv)
     assert torch.equal(o2, o1[torch.as_tensor(perm, device=DEV)])
     assert torch.equal(l2, l1[torch.as_tensor(perm, device=DEV)])
+
+
+SPLIT_CASES = [
+    # (lens, Hq, Hkv, D, ps, splits): a long pair cut into 64 pieces (two merge levels)
+    ([50000, 3], 16, 1, 128, 64, 64),
+    # one pair cut into 938 one-unit pieces (four merge levels)
+    ([60000], 8, 1, 64, 16, 4096),
+    # many short sequences per block, empty ones among them
+    ([(i * 37) % 300 for i in range(200)], 8, 2, 128, 64, 2),
+    # lengths across three orders of magnitude, page 32
+    ([1, 70000, 64, 65, 0, 9000, 128, 3000], 32, 4, 128, 32, 3),
+]
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,ps,splits", SPLIT_CASES)
+def test_split_decode_merge_tree_vs_oracle(lens, Hq, Hkv, D, ps, splits):
+    """Split-KV with many pieces per pair (partials merged in groups of 8 by the
+    last block to finish each group, level after level), many short sequences
+    and empty ones, against the fp64 oracle (sampled rows for the 200-sequence
+    batch)."""
+    q, k, v, table, kl = _paged_inputs(lens, Hq, Hkv, D, ps, seed=len(lens) + ps + splits)
+    rows = None
+    if len(lens) > 100:
+        rng = np.random.default_rng(5)
+        rows = np.array([(b, h) for b in rng.choice(len(lens), 40, replace=False) for h in range(Hq)],
+                        dtype=np.int32)
+    o, lse, _ = check_paged(q, k, v, table, kl, ps, 1.0 / np.sqrt(D), splits, rows=rows,
+                            where=f"split {len(lens)} seqs S{splits}")
+    assert torch.isfinite(o.float()).all()
+    empty = np.asarray(lens) == 0
+    if empty.any():
+        e = torch.as_tensor(np.nonzero(empty)[0], device=DEV)
+        assert torch.all(o[e] == 0) and torch.all(lse[e] == -float("inf"))
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK

@@ -8,9 +8,10 @@ built ({count, claim counter} header, then {b, qtile, h0, cost} items); the
 test copies it out and compares it with the list ``metadata_check`` derives on
 the host from the documented order: every item exactly once, each sequence's
 run in order, runs most work first, and a claim counter that shows every item
-was handed out once.  The split-decode launch order and the page-table
-coordinates (through the diagnostic entry point that runs the producers' own
-address functions) are checked the same way."""
+was handed out once.  The split-decode schedule, the split MLA decode's
+launch order and the page-table coordinates (through the diagnostic
+entry point that runs the producers' own address functions) are checked the
+same way."""
 import numpy as np
 import pytest
 import torch
@@ -123,13 +124,64 @@ def test_paged_prefill_work_list_bit_exact():
     assert claims == count + min(mc.ragged_max_tiles(len(lq), max(lq), T) * n_pairs, _sms())
 
 
-@pytest.mark.parametrize("lens_kind", ["config4", "ties"])
-def test_split_decode_launch_order(lens_kind):
-    if lens_kind == "config4":
-        L = synth.WORKLOADS["paged_decode"].seq_lengths()
+@pytest.mark.parametrize("lens_kind", ["mla_workload", "ties"])
+def test_split_mla_decode_launch_order(lens_kind):
+    """The split MLA decode's clusters take the sequences longest first."""
+    if lens_kind == "mla_workload":
+        L = synth.WORKLOADS["mla_decode"].seq_lengths()
     else:
         L = np.array([64, 4096, 64, 1, 4096, 4097, 63, 64] * 4, dtype=np.int64)
-    B, Hq, Hkv, D, ps, S = len(L), 8, 1, 64, 64, 3
+    B, Hq, ps, S = len(L), 128, 64, 3
+    table, total = synth.page_table(L, ps, 4)
+    q = synth.normal_bf16((B, Hq, 576), 1, DEV)
+    kp = synth.normal_bf16((total, 1, ps, 576), 2, DEV)
+    o = torch.empty((B, Hq, 512), dtype=torch.bfloat16, device=DEV)
+    n = rsd.attn_fwd_paged_workspace_size(B, Hq, 512, S)
+    ws = torch.full((n,), 0xA5, dtype=torch.uint8, device=DEV)
+    maxL = int(L.max())
+    rsd.attn_fwd_paged(q, kp, kp, o, None, torch.as_tensor(table, device=DEV),
+                       torch.as_tensor(L.astype(np.int32), device=DEV), page_size=ps, max_kv_len=maxL, scale=0.04,
+                       num_splits=S, workspace=ws)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    R = B * Hq
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    off = up(R * S * 512 * 4) + up(R * S * 4)
+    order = ws[off:off + 4 * B].cpu().view(torch.int32).numpy()
+    mc.check_decode_order(order, L, maxL)
+
+
+def _up(x):
+    return (x + 255) // 256 * 256
+
+
+def _split_offsets(base, B):
+    """Byte offsets of the split workspace's order and piece records, as the layout
+    states: per-sequence data [B] x 16 B, order [B], then one 32-byte record per block."""
+    order = _up(base + B * 16)
+    return order, _up(order + B * 4)
+
+
+def _pieces_from_ws(ws, order_off, segs_off, B, n_blocks):
+    order = ws[order_off:order_off + 4 * B].cpu().view(torch.int32).numpy()
+    rows = ws[segs_off:segs_off + 32 * n_blocks].cpu().view(torch.int32).numpy().reshape(n_blocks, 8)
+    return order, rows
+
+
+@pytest.mark.parametrize("lens_kind,S", [("config4", 2), ("ties_and_zeros", 3), ("one_long", 64)])
+def test_split_decode_schedule(lens_kind, S):
+    """The split-decode schedule the device writes (order and one piece per block)
+    equals the host rule, bit for bit: longest first, each pair cut into min(S, units)
+    near-equal pieces, every unit of every (sequence, KV head) in one block."""
+    if lens_kind == "config4":
+        L = synth.WORKLOADS["paged_decode"].seq_lengths()
+    elif lens_kind == "ties_and_zeros":
+        L = np.array([64, 4096, 0, 1, 4096, 4097, 63, 0, 65] * 3, dtype=np.int64)
+    else:
+        L = np.array([50000, 3], dtype=np.int64)
+    B, Hq, Hkv, D, ps = len(L), 16, 2, 128, 64
     table, total = synth.page_table(L, ps, 4)
     q = synth.normal_bf16((B, Hq, D), 1, DEV)
     kp = synth.normal_bf16((total, Hkv, ps, D), 2, DEV)
@@ -142,13 +194,39 @@ def test_split_decode_launch_order(lens_kind):
                        num_splits=S, workspace=ws)
     torch.cuda.synchronize()
     assert rsd.attn_get_device_error() == rsd.ATTN_OK
-    R = B * Hq
+    order_off, segs_off = _split_offsets(0, B)
+    order, rows = _pieces_from_ws(ws, order_off, segs_off, B, S * B * Hkv)
+    mc.check_decode_pieces(order, rows, L, Hkv, S, maxL)
 
-    def up(x):
-        return (x + 255) // 256 * 256
-    off = up(R * S * D * 4) + up(R * S * 4)
-    order = ws[off:off + 4 * B].cpu().view(torch.int32).numpy()
-    mc.check_decode_order(order, L, maxL)
+
+def test_split_decode_schedule_ragged_queries():
+    """The mixed batch's short rows: sequences of 1..qmax queries own units, the
+    chunk sequences (prefill kernel) none; the schedule follows the same rule."""
+    lens_q = [1, 3, 700, 2, 0, 1, 129, 4]
+    lens_kv = [5000, 90, 3000, 1, 64, 0, 800, 4100]
+    B, Hq, Hkv, D, ps, S = len(lens_q), 16, 2, 128, 64, 3
+    G = Hq // Hkv
+    qmax = min(4, 64 // G, max(lens_q))
+    cu_q = synth.cu_seqlens(lens_q)
+    T = int(cu_q[-1])
+    L = np.asarray(lens_kv, dtype=np.int64)
+    table, total = synth.page_table(L, ps, 5)
+    q = synth.normal_bf16((T, Hq, D), 1, DEV)
+    kp = synth.normal_bf16((total, Hkv, ps, D), 2, DEV)
+    o = torch.empty((T, Hq, D), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((B, max(lens_q), Hq), dtype=torch.float32, device=DEV)
+    n = rsd.attn_fwd_paged_prefill_workspace_size(B, max(lens_q), T, Hq, Hkv, D, S)
+    ws = torch.full((n,), 0xA5, dtype=torch.uint8, device=DEV)
+    rsd.attn_fwd_paged_prefill(q, kp, kp, o, lse, torch.as_tensor(cu_q, device=DEV), torch.as_tensor(table, device=DEV),
+                               torch.as_tensor(L.astype(np.int32), device=DEV), max_seqlen_q=max(lens_q),
+                               page_size=ps, max_kv_len=int(L.max()), scale=0.1, causal=True, workspace=ws,
+                               num_splits=S)
+    torch.cuda.synchronize()
+    assert rsd.attn_get_device_error() == rsd.ATTN_OK
+    base = rsd.attn_fwd_ragged_workspace_size(B, max(lens_q), T, Hq, Hkv)
+    order_off, segs_off = _split_offsets(base, B)
+    order, rows = _pieces_from_ws(ws, order_off, segs_off, B, S * B * Hkv)
+    mc.check_decode_pieces(order, rows, L, Hkv, S, int(L.max()), cu_q=cu_q, qmax=qmax)
 
 
 @pytest.mark.parametrize("ps", [64, 16])

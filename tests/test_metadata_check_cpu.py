@@ -110,3 +110,43 @@ def test_routed_short_sequences_have_no_items():
     extra = mc.sequence_block(0, 1, 900, 8, 2, True)
     with pytest.raises(AssertionError):
         mc.check_sequence_list(np.array(items + extra), len(items) + len(extra), lq, lkv, 8, 2, True, short_q=4)
+
+
+def _pieces(L, Hkv, S, maxL, cu_q=None, qmax=1):
+    seq = mc.decode_units(L, maxL, cu_q, qmax)
+    shift = mc.decode_sort_shift(maxL)
+    order = sorted(range(len(L)), key=lambda b: -min(mc.SORT_CAP, seq[b][0] >> shift))
+    rows = mc.decode_pieces(seq, order, Hkv, S)
+    full = np.array(rows + [(-1, 0, 0, 0, 0, 0, 0, 0)] * (S * len(L) * Hkv - len(rows)), dtype=np.int64)
+    return order, full
+
+
+@pytest.mark.parametrize("cu", [False, True])
+def test_split_pieces_rule_passes(cu):
+    L = [5000, 0, 64, 65, 1, 3000, 129, 7]
+    cu_q, qmax = (np.array([0, 1, 4, 704, 706, 706, 707, 836, 840]), 4) if cu else (None, 1)
+    order, rows = _pieces(L, 2, 3, 5000, cu_q, qmax)
+    mc.check_decode_pieces(order, rows, L, 2, 3, 5000, cu_q, qmax)
+    # pieces of one pair differ by at most one unit
+    for r in rows[rows[:, 0] >= 0]:
+        n = mc.decode_units(L, 5000, cu_q, qmax)[r[0] // 2][0]
+        assert (r[2] - r[1]) in (n // r[4], -(-n // r[4]))
+
+
+def test_split_pieces_out_of_order_fails():
+    L = [5000, 64, 3000]
+    order, rows = _pieces(L, 2, 3, 5000)
+    with pytest.raises(AssertionError):
+        mc.check_decode_pieces([order[1], order[0], order[2]], rows, L, 2, 3, 5000)
+
+
+@pytest.mark.parametrize("field,delta", [(1, 1), (2, -1), (3, 1), (4, 1)])
+def test_split_pieces_altered_record_fails(field, delta):
+    """A piece that starts or ends one unit off (a gap or an overlap), or points at
+    the wrong slots or piece count, is rejected."""
+    L = [5000, 64, 3000]
+    order, rows = _pieces(L, 2, 3, 5000)
+    bad = rows.copy()
+    bad[1, field] += delta
+    with pytest.raises(AssertionError):
+        mc.check_decode_pieces(order, bad, L, 2, 3, 5000)
