@@ -69,12 +69,16 @@ int setup_device(int* dev_out, int* sms_out) {
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(b2::prefill_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::PrefillCfg<128>::SMEM);
-        const void* decode_kernels[6] = {(const void*)b2::decode_gqa_kernel<64, 1>, (const void*)b2::decode_gqa_kernel<64, 2>,
+        const void* decode_kernels[8] = {(const void*)b2::decode_gqa_kernel<64, 1>, (const void*)b2::decode_gqa_kernel<64, 2>,
                                          (const void*)b2::decode_gqa_kernel<64, 4>, (const void*)b2::decode_gqa_kernel<128, 1>,
-                                         (const void*)b2::decode_gqa_kernel<128, 2>, (const void*)b2::decode_gqa_kernel<128, 4>};
-        for (int i = 0; i < 6 && e == cudaSuccess; ++i)
-            e = cudaFuncSetAttribute(decode_kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     i < 3 ? b2::DecodeCfg<64>::SMEM : b2::DecodeCfg<128>::SMEM);
+                                         (const void*)b2::decode_gqa_kernel<128, 2>, (const void*)b2::decode_gqa_kernel<128, 4>,
+                                         (const void*)b2::decode_gqa_kernel<64, 1, 6>,
+                                         (const void*)b2::decode_gqa_kernel<128, 1, 6>};
+        const int decode_smem[8] = {b2::DecodeCfg<64>::SMEM,     b2::DecodeCfg<64>::SMEM,  b2::DecodeCfg<64>::SMEM,
+                                    b2::DecodeCfg<128>::SMEM,    b2::DecodeCfg<128>::SMEM, b2::DecodeCfg<128>::SMEM,
+                                    b2::DecodeCfg<64, 6>::SMEM, b2::DecodeCfg<128, 6>::SMEM};
+        for (int i = 0; i < 8 && e == cudaSuccess; ++i)
+            e = cudaFuncSetAttribute(decode_kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize, decode_smem[i]);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(b2::decode_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      b2::MlaTcCfg::SMEM);
@@ -260,8 +264,15 @@ int launch_decode_schedule(DecodeParams& dp, char* wsb, const SplitWs& w, int64_
 }
 
 // Launches the GQA decode kernel with RT 16-row m-tiles (1, 2 or 4): grid
-// (1, Hkv, B) without splits, one block per scheduled piece with them.
-int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, cudaStream_t st) {
+// (1, Hkv, B) without splits, one block per scheduled piece with them.  A
+// launch of at most one block per SM gets the 6-stage ring (RT 1).
+int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, int sms, cudaStream_t st) {
+    const int64_t blocks = (int64_t)grid.x * grid.y * grid.z;
+    if (RT == 1 && blocks <= sms) {
+        if (D == 128) b2::decode_gqa_kernel<128, 1, 6><<<grid, 160, b2::DecodeCfg<128, 6>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<64, 1, 6><<<grid, 160, b2::DecodeCfg<64, 6>::SMEM, st>>>(dp);
+        return launch_status();
+    }
     if (D == 128) {
         if (RT == 1) b2::decode_gqa_kernel<128, 1><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
         else if (RT == 2) b2::decode_gqa_kernel<128, 2><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
@@ -728,9 +739,9 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         dp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
         if (num_splits > 1) {
             if (int e = launch_decode_schedule(dp, wsb, wl.sw, n_cta, max_kv_len, st)) return e;
-            if (int e = launch_decode_gqa(dp, D, RT, dim3((unsigned)n_cta, 1, 1), st)) return e;
+            if (int e = launch_decode_gqa(dp, D, RT, dim3((unsigned)n_cta, 1, 1), sms, st)) return e;
         } else {
-            if (int e = launch_decode_gqa(dp, D, RT, dim3(1, Hkv, B), st)) return e;
+            if (int e = launch_decode_gqa(dp, D, RT, dim3(1, Hkv, B), sms, st)) return e;
         }
     }
 
@@ -1002,9 +1013,9 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     if (num_splits > 1) {
         const SplitWs sw = split_ws_layout(0, B, R, 1, Dv, num_splits);
         if (int e = launch_decode_schedule(dp, wsb, sw, n_cta, max_kv_len, st)) return e;
-        return launch_decode_gqa(dp, Dqk, 1, dim3((unsigned)n_cta, 1, 1), st);
+        return launch_decode_gqa(dp, Dqk, 1, dim3((unsigned)n_cta, 1, 1), sms, st);
     }
-    return launch_decode_gqa(dp, Dqk, 1, dim3(1, Hkv, B), st);
+    return launch_decode_gqa(dp, Dqk, 1, dim3(1, Hkv, B), sms, st);
 }
 
 // ------------------------------------------------------------------ merge

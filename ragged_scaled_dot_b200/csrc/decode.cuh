@@ -263,12 +263,15 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const __grid_cons
 // of the warps of one m-tile are combined through the stage of the last chunk,
 // each row's weights computed once.  RT = 1 without cu_q is plain decode.
 // ===========================================================================
-template <int D>
+// NST stages of K/V: 3 lets two blocks share an SM; 6 is for launches with at most
+// one block per SM, which then keep twice the bytes in flight.
+template <int D, int NST_ = 3>
 struct DecodeCfg {
     static constexpr int NCB = D / 64;                  // 64-wide column blocks
     static constexpr uint32_t BLK = 64 * 128;           // one column block of a chunk
     static constexpr uint32_t CHUNK = NCB * BLK;        // K (or V) bytes of a chunk
-    static constexpr int NST = 3;
+    static constexpr int NST = NST_;
+    static_assert(NST >= 2 && 16 * NST + 4 <= 128, "full and empty barriers and the abort flag fit the barrier area");
     static constexpr uint32_t STAGE = 2 * CHUNK;        // K then V
     static constexpr uint32_t BAR_OFF = NST * STAGE;
     // the page ids of the piece (K table, then V table when it has its own), read by the
@@ -368,9 +371,9 @@ __device__ __forceinline__ void decode_merge_up(const DecodeParams& p, const Dec
     }
 }
 
-template <int D, int RT>
-__global__ void __launch_bounds__(160, 2) decode_gqa_kernel(const __grid_constant__ DecodeParams p) {
-    using C = DecodeCfg<D>;
+template <int D, int RT, int NST_ = 3>
+__global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(const __grid_constant__ DecodeParams p) {
+    using C = DecodeCfg<D, NST_>;
     constexpr int NST = C::NST;
     constexpr int KW = 16 * RT;  // keys of every chunk one compute warp owns
     static_assert(RT == 1 || RT == 2 || RT == 4, "m-tiles");
