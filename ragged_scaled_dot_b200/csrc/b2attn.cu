@@ -285,19 +285,21 @@ int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, int sms,
     return launch_status();
 }
 
-// GQA decode maps over a pool: (d, slot, head, page), 64-column boxes of one
-// page's min(page_size, 64) rows.
+// GQA decode maps over a pool: (column in block, slot, 64-column block, head,
+// page), one box per page: its min(page_size, 64) rows in every column block,
+// landing in shared memory as [column block][rows][128 B].
 int encode_decode_pool_maps(DecodeParams& dp, const void* k_pool, const void* v_pool, int Dqk, int Dv, int page_size,
                             int Hkv, int64_t num_pages, const int64_t k_pool_strides[3],
                             const int64_t v_pool_strides[3]) {
     const int box_rows = page_size < 64 ? page_size : 64;
-    const uint32_t box[4] = {64, (uint32_t)box_rows, 1, 1};
-    const uint64_t dk[4] = {(uint64_t)Dqk, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
-    const int64_t sk[3] = {k_pool_strides[1], k_pool_strides[2], k_pool_strides[0]};
-    if (encode_4d(&dp.tm_k, k_pool, dk, sk, box)) return ATTN_ERR_INVALID_ARG;
-    const uint64_t dv[4] = {(uint64_t)Dv, (uint64_t)page_size, (uint64_t)Hkv, (uint64_t)num_pages};
-    const int64_t sv[3] = {v_pool_strides[1], v_pool_strides[2], v_pool_strides[0]};
-    if (encode_4d(&dp.tm_v, v_pool, dv, sv, box)) return ATTN_ERR_INVALID_ARG;
+    const uint32_t bk[5] = {64, (uint32_t)box_rows, (uint32_t)(Dqk / 64), 1, 1};
+    const uint64_t dk[5] = {64, (uint64_t)page_size, (uint64_t)(Dqk / 64), (uint64_t)Hkv, (uint64_t)num_pages};
+    const int64_t sk[4] = {k_pool_strides[1] * 2, 128, k_pool_strides[2] * 2, k_pool_strides[0] * 2};
+    if (encode_5d(&dp.tm_k, k_pool, dk, sk, bk)) return ATTN_ERR_INVALID_ARG;
+    const uint32_t bv[5] = {64, (uint32_t)box_rows, (uint32_t)(Dv / 64), 1, 1};
+    const uint64_t dv[5] = {64, (uint64_t)page_size, (uint64_t)(Dv / 64), (uint64_t)Hkv, (uint64_t)num_pages};
+    const int64_t sv[4] = {v_pool_strides[1] * 2, 128, v_pool_strides[2] * 2, v_pool_strides[0] * 2};
+    if (encode_5d(&dp.tm_v, v_pool, dv, sv, bv)) return ATTN_ERR_INVALID_ARG;
     dp.box_rows = box_rows;
     return ATTN_OK;
 }

@@ -45,7 +45,9 @@ constexpr int kMergeFan = 8;     // partials merged by one block
 constexpr int kMergeLevels = 4;  // up to kMergeFan^4 pieces per pair
 
 struct DecodeParams {
-    CUtensorMap tm_k;  // 4D (d, slot, head, page), 128B swizzle, box (64, min(ps,64), 1, 1)
+    // GQA: 5D (column in block, slot, 64-column block, head, page), 128B swizzle, box
+    // (64, min(ps, 64), D / 64, 1, 1); MLA: the 5D maps of decode_mla.cuh
+    CUtensorMap tm_k;
     CUtensorMap tm_v;
     const __nv_bfloat16* q;
     int64_t q_bs, q_hs;  // (batch, head) element strides; with cu_q: (token, head)
@@ -123,14 +125,17 @@ __device__ __forceinline__ uint32_t decode_chunk_bytes(const DecodeParams& p, in
 }
 
 // Issues the K and V TMA loads of the chunk from t0 for kv head g of sequence b:
-// rows [r, r + box_rows) come from one page (NB = 64 / box_rows boxes).  All
-// page ids of the chunk are read before any box is issued, so their latencies
-// overlap (each TMA issue is ordered after the reads before it; one thread
-// reading them box by box could not keep a small batch's few blocks streaming),
-// and with one page table for K and V the V boxes reuse the K boxes' ids.
+// rows [r, r + box_rows) come from one page (NB = 64 / box_rows boxes), each box
+// all column blocks of those rows, landing at dst + i * (ncol_blocks * box_rows *
+// 128) as [column block][rows][128 B] (for box_rows 64: the [column block][64
+// rows] tile).  All page ids of the chunk are read before any box is issued, so
+// their latencies overlap (each TMA issue is ordered after the reads before it;
+// one thread reading them box by box could not keep a small batch's few blocks
+// streaming), and with one page table for K and V the V boxes reuse the K
+// boxes' ids.
 template <int NB>
 __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t dst_k, uint32_t dst_v, uint32_t bar,
-                                                int b, int g, int t0, int hi, int ncol_blocks, uint32_t block_bytes,
+                                                int b, int g, int t0, int hi, int ncol_blocks,
                                                 const volatile int* ids_k, const volatile int* ids_v, int p0, int nids) {
     const int R = p.box_rows;
     const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
@@ -151,6 +156,7 @@ __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t 
                                                        : page_lookup(p.v_page_table, p.v_pt_stride, b, t,
                                                                      p.page_size)));
     }
+    const uint32_t box_bytes = (uint32_t)(ncol_blocks * R) * 128u;
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
         const int t = t0 + i * R;
@@ -159,12 +165,17 @@ __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t 
             const int pk = page_checked(idk[i], p.num_pages);
             const int pv = shared_table ? pk : page_checked(idv[i], p.num_pages);
             const int slot = page_slot(t, p.page_size);
-            for (int cb = 0; cb < ncol_blocks; ++cb) {
-                tma_load_4d(dst_k + cb * block_bytes + (uint32_t)(i * R) * 128u, &p.tm_k, bar, cb * 64, slot, g, pk);
-                tma_load_4d(dst_v + cb * block_bytes + (uint32_t)(i * R) * 128u, &p.tm_v, bar, cb * 64, slot, g, pv);
-            }
+            tma_load_5d(dst_k + i * box_bytes, &p.tm_k, bar, 0, slot, 0, g, pk);
+            tma_load_5d(dst_v + i * box_bytes, &p.tm_v, bar, 0, slot, 0, g, pv);
         }
     }
+}
+
+// Byte offset of key row k of a chunk's K (or V) tile, column block 0: page box
+// k / R of NCB column blocks of R rows (R = 2^lR, at least 8), row k % R.  The
+// 128-byte swizzle of the row is (k & 7), as each box starts on 1 KB.
+__device__ __forceinline__ uint32_t decode_row_off(int k, int lR, int ncb) {
+    return ((uint32_t)((k >> lR) * ncb) << (lR + 7)) + ((uint32_t)(k & ((1 << lR) - 1)) << 7);
 }
 
 // ===========================================================================
@@ -268,7 +279,7 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const __grid_cons
 template <int D, int NST_ = 3>
 struct DecodeCfg {
     static constexpr int NCB = D / 64;                  // 64-wide column blocks
-    static constexpr uint32_t BLK = 64 * 128;           // one column block of a chunk
+    static constexpr uint32_t BLK = 64 * 128;           // one column block of a chunk (64 rows of 128 B)
     static constexpr uint32_t CHUNK = NCB * BLK;        // K (or V) bytes of a chunk
     static constexpr int NST = NST_;
     static_assert(NST >= 2 && 16 * NST + 4 <= 128, "full and empty barriers and the abort flag fit the barrier area");
@@ -474,20 +485,20 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
                 const uint32_t dst = sb + st * C::STAGE;
                 switch (64 / p.box_rows) {
                     case 1:
-                        decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK,
-                                           ids_k, ids_v, p0, nids);
+                        decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
+                                           p0, nids);
                         break;
                     case 2:
-                        decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK,
-                                           ids_k, ids_v, p0, nids);
+                        decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
+                                           p0, nids);
                         break;
                     case 4:
-                        decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK,
-                                           ids_k, ids_v, p0, nids);
+                        decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
+                                           p0, nids);
                         break;
                     default:
-                        decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, C::BLK,
-                                           ids_k, ids_v, p0, nids);
+                        decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
+                                           p0, nids);
                         break;
                 }
             }
@@ -553,6 +564,17 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
         float oacc[D / 8][4];
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
+        // this lane's ldmatrix rows in every chunk: keys kbase + 16 kg + (0 or 8) + lane % 8
+        // of the QK (K) and PV (V) fragments, as offsets into the page-box layout; their
+        // 128-byte swizzle is lane % 8
+        const int lR = 31 - __clz(p.box_rows);
+        const uint32_t cbs = 128u << lR;  // bytes per column block of a page box
+        uint32_t row_k[RT], row_v[RT];
+#pragma unroll
+        for (int kg = 0; kg < RT; ++kg) {
+            row_k[kg] = decode_row_off(kbase + 16 * kg + (((lane >> 3) >> 1) << 3) + (lane & 7), lR, C::NCB);
+            row_v[kg] = decode_row_off(kbase + 16 * kg + (((lane >> 3) & 1) << 3) + (lane & 7), lR, C::NCB);
+        }
 
         for (int k = 0; k < n_chunks; ++k) {
             const int st = k % NST;
@@ -572,7 +594,8 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
                         const int rem = i % (C::NCB * 8);
                         const int cb = rem / 8, ch = rem % 8;
                         if (rr >= nvalid)
-                            *reinterpret_cast<uint4*>(vg + cb * C::BLK + rr * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(vg + decode_row_off(rr, lR, C::NCB) + cb * cbs + ch * 16) =
+                                make_uint4(0, 0, 0, 0);
                     }
                     __syncwarp();
                 }
@@ -587,16 +610,15 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
 #pragma unroll
                     for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.f;
                 {
-                    const int mat = lane >> 3, rr = lane & 7;
+                    const int mat = lane >> 3, sw = lane & 7;
 #pragma unroll
                     for (int kg = 0; kg < RT; ++kg) {
-                        const int key = kbase + 16 * kg + ((mat >> 1) << 3) + rr;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const int cb = kk >> 2;
-                            const int dcol = (kk & 3) * 16 + ((mat & 1) << 3);
+                            const uint32_t chunk16 = (uint32_t)((((kk & 3) << 1) | (mat & 1)) ^ sw);
                             uint32_t b0, b1, b2, b3;
-                            ldsm_x4(sK + cb * C::BLK + sw128_offset(key, dcol), b0, b1, b2, b3);
+                            ldsm_x4(sK + row_k[kg] + cb * cbs + (chunk16 << 4), b0, b1, b2, b3);
                             float (&a0)[4] = (kTwoChains && (kk & 1)) ? sacc2[2 * kg] : sacc[2 * kg];
                             float (&a1)[4] = (kTwoChains && (kk & 1)) ? sacc2[2 * kg + 1] : sacc[2 * kg + 1];
                             mma_bf16_16816(a0, qa[kk], b0, b1);
@@ -657,7 +679,7 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
                     }
                 }
                 // O += P V over this warp's keys, 16 keys per k-step
-                const int mat = lane >> 3, rr = lane & 7;
+                const int mat = lane >> 3, sw = lane & 7;
 #pragma unroll
                 for (int kg = 0; kg < RT; ++kg) {
                     uint32_t pa[4];
@@ -665,13 +687,12 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
                     pa[1] = pack_bf16(sacc[2 * kg][2], sacc[2 * kg][3]);
                     pa[2] = pack_bf16(sacc[2 * kg + 1][0], sacc[2 * kg + 1][1]);
                     pa[3] = pack_bf16(sacc[2 * kg + 1][2], sacc[2 * kg + 1][3]);
-                    const int key = kbase + 16 * kg + ((mat & 1) << 3) + rr;
 #pragma unroll
                     for (int nd = 0; nd < D / 16; ++nd) {
                         const int cb = nd >> 2;
-                        const int dcol = (nd & 3) * 16 + ((mat >> 1) << 3);
+                        const uint32_t chunk16 = (uint32_t)((((nd & 3) << 1) | (mat >> 1)) ^ sw);
                         uint32_t v0, v1, v2, v3;
-                        ldsm_x4_t(sV + cb * C::BLK + sw128_offset(key, dcol), v0, v1, v2, v3);
+                        ldsm_x4_t(sV + row_v[kg] + cb * cbs + (chunk16 << 4), v0, v1, v2, v3);
                         mma_bf16_16816(oacc[2 * nd], pa, v0, v1);
                         mma_bf16_16816(oacc[2 * nd + 1], pa, v2, v3);
                     }
