@@ -347,9 +347,10 @@ size_t attn_fwd_paged_workspace_size(int B, int Hq, int Dv, int num_splits);
  * stay a small fraction of the KV bytes streamed ("cuDNN Frontend v1.31.0
  * Release Notes", "SDPA: paged KV, split-KV, and engine selection": split
  * selection from the physical launch capacity and the ragged work, not from a
- * dense envelope).  A small batch (at most two waves of blocks) gets the
- * count whose last wave is fullest.  Host-only arithmetic; the choice never
- * changes results beyond rounding.
+ * dense envelope).  GQA batches that fit one wave of blocks (two per SM)
+ * get the count that fills that wave, or one block per SM for whole-page
+ * boxes of 64 rows over caches of at most 8192 keys.  Host-only arithmetic;
+ * the choice never changes results beyond rounding.
  */
 int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_kv_len,
                               int page_size, int num_sms);

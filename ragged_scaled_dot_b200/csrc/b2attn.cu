@@ -833,6 +833,21 @@ int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_k
     } else {
         const int64_t ctas_per_split = (int64_t)Hkv * B;
         const int64_t slots = (int64_t)num_sms * 2;
+        if (ctas_per_split <= slots) {
+            // the batch fits one wave of blocks (two per SM) without splits: the count that
+            // gives the most blocks still in one wave (b 32 / Hkv 4 / 4096 keys, page 16:
+            // 2 splits 58.4 us against 85.1 with 1 and 81.9 with 3; b 8: 8 splits 29.3 us
+            // against 41.5 with 3; b 64: 1 split 91.7 us against 112 with 2). With whole-page
+            // boxes of 64 rows and short caches, one block per SM with the deep ring wins
+            // instead (b 32, page 64: 1 split 49.7 us against 55.7 with 2; at 16384 keys 2
+            // splits win, 167 against 176 us)
+            int64_t s = slots / ctas_per_split;
+            if (page_size >= 64 && max_kv_len <= 8192 && ctas_per_split <= num_sms) s = num_sms / ctas_per_split;
+            const int64_t units = ((int64_t)max_kv_len + 63) / 64;
+            if (s > units) s = units;
+            if (s > 512) s = 512;
+            return (int)(s < 1 ? 1 : s);
+        }
         // about four waves of CTAs over the two resident CTAs per SM (longest sequences
         // first; measured best on the 128-sequence GQA workload against 8 and 16)
         s_balance = (4 * slots + ctas_per_split - 1) / ctas_per_split;
@@ -847,27 +862,6 @@ int attn_paged_suggest_splits(int B, int Hq, int Hkv, int Dqk, int Dv, int max_k
     if (s > max_pages) s = max_pages;
     if (s > 64) s = 64;
     if (s < 1) s = 1;
-    if (!mla) {
-        // a small batch (at most two waves of CTAs): a last wave that is only partly full
-        // costs as much as a full one, so take the count with the fewest waves per unit of
-        // work, fewer splits on a tie (b 32, Hkv 4, 4096 keys, page 16: 2 splits measured
-        // 72 us against 102 with 3 and 104 with 1)
-        const int64_t ctas_per_split = (int64_t)Hkv * B;
-        const int64_t slots = (int64_t)num_sms * 2;
-        if (ctas_per_split * s <= 2 * slots) {
-            int64_t best = 1;
-            double best_cost = 1e30;
-            for (int64_t c = 1; c <= s; ++c) {
-                const double waves = (double)((ctas_per_split * c + slots - 1) / slots);
-                const double cost = waves / (double)c + 0.01 * (double)c;
-                if (cost < best_cost) {
-                    best_cost = cost;
-                    best = c;
-                }
-            }
-            s = best;
-        }
-    }
     return (int)s;
 }
 
