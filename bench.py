@@ -615,6 +615,8 @@ def run_ours(args):
         extras.append(make_paged_prefill(torch, rsd, synth, dev, off)[0])
         mla, _ = make_paged(torch, rsd, synth, dev, off, "mla_decode", num_sms)
         extras.append(mla)
+        small, _ = make_paged(torch, rsd, synth, dev, off, "decode_small_batch", num_sms)
+        extras.append(small)
         for subset in ("all", "short", "chunks"):
             extras.append(make_mixed(torch, rsd, synth, dev, off, num_sms, subset))
     torch.cuda.synchronize()
@@ -704,6 +706,11 @@ def run_ours(args):
         v, ms, roof = part_summary(part, bound)
         extra_out[part.name] = {"value": round(v, 2), "unit": part.unit, "ms_per_step": round(ms, 4),
                                 "roofline": roof, **part.info}
+        if part.name == "decode_small_batch":
+            # the pages print a latency for this shape: 44 us for cuDNN's decode engine (GPU not
+            # named), context rather than a target
+            extra_out[part.name]["us_per_call"] = round(ms * 1e3, 1)
+            extra_out[part.name]["pages_decode_engine_us"] = 44.0
         if part.name == "mla_decode":
             tflops = part.info["flop_per_step"] / 1e12 / (ms / 1e3)
             extra_out[part.name]["tflops"] = round(tflops, 2)
@@ -832,7 +839,8 @@ def main():
     ap.add_argument("--part-gap", type=float, default=2.0,
                     help="seconds of idle GPU before each part after the first")
     ap.add_argument("--only", choices=["ragged_prefill", "paged_decode", "dense_prefill", "paged_prefill",
-                                       "mla_decode", "mixed_batch", "mixed_short_rows", "mixed_chunks"],
+                                       "mla_decode", "decode_small_batch", "mixed_batch", "mixed_short_rows",
+                                       "mixed_chunks"],
                     help="profiling: time one part only and print its own line")
     ap.add_argument("--batch", type=int, default=0, help="profiling: override the part's batch size")
     args = ap.parse_args()

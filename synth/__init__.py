@@ -114,6 +114,11 @@ WORKLOADS = {
         "paged_decode", "paged", seed=4, B=128, Hq=64, Hkv=8, Dqk=128, Dv=128,
         len_range=(1024, 32768), page_size=64, causal=False,
         notes="paged decode B=128 kv U[1024, 32768] page 64, H=64/8 D=128"),
+    "decode_small_batch": Workload(
+        "decode_small_batch", "paged", seed=8, B=32, Hq=64, Hkv=4, Dqk=128, Dv=128,
+        len_range=(4096, 4096), page_size=16, causal=False,
+        notes="paged decode b=32, 4096 cached keys each, page 16, H=64/4 D=128 (the shape of the "
+              "decode latencies in 'cuDNN Frontend v1.30.0 Release Notes', 'New: decode tiles')"),
     "paged_prefill": Workload(
         "paged_prefill", "paged", seed=6, B=16, Hq=32, Hkv=8, Dqk=128, Dv=128,
         lengths=(1024,), len_range=(8192, 65536), page_size=64, causal=True,

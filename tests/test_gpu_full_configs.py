@@ -71,7 +71,7 @@ def test_ragged_prefill_full_size():
                          torch.as_tensor(rows[:, 2].astype(np.int64), device=DEV), h], l_ref, "ragged full")
 
 
-@pytest.mark.parametrize("name", ["paged_decode", "mla_decode"])
+@pytest.mark.parametrize("name", ["paged_decode", "mla_decode", "decode_small_batch"])
 def test_paged_decode_full_size(name):
     w = synth.WORKLOADS[name]
     L = w.seq_lengths()
@@ -89,7 +89,7 @@ def test_paged_decode_full_size(name):
     assert rsd.attn_get_device_error() == rsd.ATTN_OK
     assert not torch.isnan(o).any()
     rng = np.random.default_rng(2)
-    if name == "paged_decode":
+    if name in ("paged_decode", "decode_small_batch"):
         bs = rng.choice(w.B, 24, replace=False)
         rows = np.array([(b, h) for b in bs for h in range(w.Hq)], dtype=np.int32)
     else:
