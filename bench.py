@@ -42,12 +42,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the full launch.  None when the kernel changed after the counters were taken
 # or has no capture.
 #   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.0404 / 1.0611 GB)
-#   paged_decode: per K/V byte, batch 32 (2.6866 / 2.6734 GB)
+#   paged_decode: per K/V byte, batch 16, 2 splits (1.3666 / 1.3589 GB)
 #   mla_decode: per K/V byte, batch 8 (0.3439 / 0.3355 GB; the partials grow with the
 #     batch like the K/V bytes)
 #   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.6837 / 0.6345 GB)
 #   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7045 / 0.6711 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0049, "mla_decode": 1.0262, "paged_prefill": 1.0760,
+TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0057, "mla_decode": 1.0262, "paged_prefill": 1.0760,
                  "dense_prefill": 1.0497}
 
 
@@ -324,7 +324,8 @@ def make_mixed(torch, rsd, synth, dev, seed_offset, num_sms, subset="all"):
     lse = torch.empty((T, w.Hq), dtype=torch.float32, device=dev)
     maxL = int(L.max())
     n_short = int(np.sum((lq >= 1) & (lq <= 4)))
-    S = rsd.attn_paged_suggest_splits(max(1, n_short), w.Hq, w.Hkv, w.Dqk, w.Dv, maxL, w.page_size, num_sms)
+    # the split count of the short rows (none to split without them)
+    S = rsd.attn_paged_suggest_splits(n_short, w.Hq, w.Hkv, w.Dqk, w.Dv, maxL, w.page_size, num_sms) if n_short else 1
     ws = torch.empty(rsd.attn_fwd_paged_prefill_workspace_size(w.B, smax, T, w.Hq, w.Hkv, w.Dqk, S),
                      dtype=torch.uint8, device=dev)
     cud = torch.as_tensor(cu_q, device=dev)
