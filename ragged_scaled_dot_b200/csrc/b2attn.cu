@@ -934,11 +934,19 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     // rows per TMA box: one page, at most 64 keys
     const int box_rows = page_size < 64 ? page_size : 64;
     if (mla) {
-        // (column in block, row in page, 64-column block, head, page); 3 blocks per K load, 4 per V load
-        const uint64_t dk[5] = {64, (uint64_t)page_size, 9, (uint64_t)Hkv, (uint64_t)num_pages};
-        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, k_pool_strides[2] * 2, k_pool_strides[0] * 2};
-        const uint32_t bk[5] = {64, (uint32_t)box_rows, (uint32_t)b2::MlaTcCfg::KB, 1, 1};
+        // K: (column in block, row in 8-row group, 64-column block, 8-row group of the pool, head),
+        // one box per page box of R rows and all 9 column blocks, landing group-major; the pool's
+        // page stride must be a whole number of 8-row groups
+        const int64_t gk = k_pool_strides[0] / (8 * k_pool_strides[1]);
+        if (k_pool_strides[0] % (8 * k_pool_strides[1]) != 0 || gk < page_size / 8 ||
+            (int64_t)num_pages * gk >= ((int64_t)1 << 31))
+            return ATTN_ERR_UNSUPPORTED;
+        const uint64_t dk[5] = {64, 8, 9, (uint64_t)(num_pages * gk), (uint64_t)Hkv};
+        const int64_t sk[4] = {k_pool_strides[1] * 2, 128, 8 * k_pool_strides[1] * 2, k_pool_strides[2] * 2};
+        const uint32_t bk[5] = {64, 8, 9, (uint32_t)(box_rows / 8), 1};
         if (encode_5d(&dp.tm_k, k_pool, dk, sk, bk)) return ATTN_ERR_INVALID_ARG;
+        dp.groups_per_page = (int)gk;
+        // V: (column in block, row in page, 64-column block, head, page), 8 value blocks per load
         const uint64_t dv[5] = {64, (uint64_t)page_size, 8, (uint64_t)Hkv, (uint64_t)num_pages};
         const int64_t sv[4] = {v_pool_strides[1] * 2, 128, v_pool_strides[2] * 2, v_pool_strides[0] * 2};
         const uint32_t bv[5] = {64, (uint32_t)box_rows, (uint32_t)b2::MlaTcCfg::VB, 1, 1};

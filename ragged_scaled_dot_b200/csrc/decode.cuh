@@ -46,7 +46,9 @@ constexpr int kMergeLevels = 4;  // up to kMergeFan^4 pieces per pair
 
 struct DecodeParams {
     // GQA: 5D (column in block, slot, 64-column block, head, page), 128B swizzle, box
-    // (64, min(ps, 64), D / 64, 1, 1); MLA: the 5D maps of decode_mla.cuh
+    // (64, min(ps, 64), D / 64, 1, 1); MLA: K (column in block, row in 8-row group,
+    // column block, 8-row group, head), box (64, 8, 9, min(ps, 64) / 8, 1), and V as for GQA
+    // with 8 column blocks
     CUtensorMap tm_k;
     CUtensorMap tm_v;
     const __nv_bfloat16* q;
@@ -67,6 +69,7 @@ struct DecodeParams {
     int causal;
     int B, Hq, Hkv, G;
     int page_size, box_rows;  // rows per TMA box: min(page_size, chunk keys)
+    int groups_per_page;      // MLA K map: 8-row groups per page stride (group-major boxes)
     int64_t num_pages;
     int max_kv_len;
     int num_splits;

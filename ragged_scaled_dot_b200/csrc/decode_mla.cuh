@@ -22,10 +22,11 @@
 //     writes O / 1/l (or the fp32 split partial).
 //
 // Loads: a page box covers R = min(page_size, 64) rows and several adjacent
-// 64-column blocks of each row (5D tensor map: column in block, row, block,
-// head, page): all 9 blocks of a page's K rows per score-CTA load and the 8
-// value blocks per value-CTA load, so each TMA request reads a whole cache
-// row.  Measured on B200, one SM streams about 220 GB/s with such boxes but
+// 64-column blocks of each row: all 9 blocks of a page's K rows per score-CTA
+// load and the 8 value blocks per value-CTA load, so each TMA request reads a
+// whole cache row.  The K boxes land group-major ([8-row group][column block]
+// [8 rows][128 B]), so every ring slot is one uniform N = 64 MMA operand and
+// two adjacent slots one N = 128 operand.  Measured on B200, one SM streams about 220 GB/s with such boxes but
 // only 60 GB/s with boxes of one 64-column block (128-byte pieces of 1152-byte
 // rows) and 80 GB/s with three; the smaller boxes left the kernel load-bound.
 // Both CTAs stream the same pages (the second read hits L2); page ids are
@@ -46,8 +47,8 @@ struct MlaTcCfg {
     static constexpr uint32_t BLK = 64u * 128u;          // 64 rows x 64 bf16 columns (R = 64)
     static constexpr int KB = 9;                         // K column blocks per score-CTA load (9 per row)
     static constexpr int VB = 8;                         // V column blocks per value-CTA load (8 per row)
-    static constexpr int KLOADS = 9 / KB, VLOADS = 8 / VB;  // loads per chunk
-    static constexpr uint32_t KSLOT = KB * BLK;          // [page][KB blocks][R rows][128 B]
+    static constexpr int KLOADS = 9 / KB, VLOADS = 8 / VB;  // loads per chunk (K: one, group-major)
+    static constexpr uint32_t KSLOT = KB * BLK;          // 64 K rows group-major: [8 groups][9 blocks][8 rows][128 B]
     static constexpr uint32_t VSLOT = VB * BLK;          // [page][VB blocks][R rows][128 B]
     static constexpr int RK = 3;                         // score CTA ring (loads in flight)
     static constexpr int RV = 2;                         // value CTA ring
@@ -87,6 +88,7 @@ struct MlaTcCfg {
 static_assert(MlaTcCfg::MSG_BYTES <= MlaTcCfg::PSLOT, "message slot");
 static_assert(MlaTcCfg::SMEM <= 232448, "shared memory");
 static_assert(MlaTcCfg::RK <= 8 && MlaTcCfg::RV <= 8, "barrier area");
+static_assert(MlaTcCfg::KB == 9 && MlaTcCfg::KLOADS == 1, "one group-major K load per chunk");
 static_assert(9 % MlaTcCfg::KB == 0 && 8 % MlaTcCfg::VB == 0 && MlaTcCfg::VB % 2 == 0 && MlaTcCfg::VLOADS <= 2, "blocks");
 
 // Page ids of the np = 64 / R page boxes of the chunk starting at key t0.  The
@@ -106,6 +108,26 @@ __device__ __forceinline__ uint32_t mla_fetch_pages(const DecodeParams& p, const
         }
     }
     return live;
+}
+
+// The score CTA's K load of a chunk: box i (R rows, all 9 column blocks) lands
+// at dst + i * R * 1152 group-major, [8-row group][column block][8 rows][128 B],
+// so a slot's 64 rows are 8 groups 9 KB apart whatever the page size.  Boxes
+// past the split, or with an out-of-range page id (recorded as an input
+// error), start at a negative group coordinate and read as zeros.
+__device__ __forceinline__ void mla_issue_k(const DecodeParams& p, uint32_t dst, uint32_t bar, int t0, int np,
+                                            const int (&pg)[4], uint32_t live) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (i < np) {
+            int grp = -(p.box_rows / 8);
+            if ((live >> i) & 1u) {
+                const int page = page_checked(pg[i], p.num_pages);
+                if (page >= 0) grp = page_group(page, page_slot(t0 + i * p.box_rows, p.page_size), p.groups_per_page);
+            }
+            tma_load_5d(dst + (uint32_t)(i * p.box_rows) * 1152u, &p.tm_k, bar, 0, 0, 0, grp, 0);
+        }
+    }
 }
 
 // One load of `nblk` column blocks starting at block blk0 for every page box
@@ -217,8 +239,7 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
                         break;
                     }
                     mbar_arrive_expect_tx(sBar + C::B_KFULL + 8 * st, C::KSLOT);
-                    mla_issue(p, &p.tm_k, sb + C::S_RING + st * C::KSLOT, sBar + C::B_KFULL + 8 * st, C::KB * t, C::KB,
-                              t0, np, pc, lc);
+                    mla_issue_k(p, sb + C::S_RING + st * C::KSLOT, sBar + C::B_KFULL + 8 * st, t0, np, pc, lc);
                     ++ki;
                 }
             }
@@ -226,40 +247,39 @@ __global__ void __launch_bounds__(320, 1) decode_mla_tc_kernel(const __grid_cons
             for (int kk = max(0, ki - C::RK); kk < ki; ++kk)
                 mbar_wait(sBar + C::B_KFULL + 8 * (kk % C::RK), (kk / C::RK) & 1, nullptr, 100000000ull);
         } else if (warp == 1 && lane == 0) {
-            const uint32_t IDESC = idesc_bf16_f32(128, R, false);
-            const SmemDesc dK = smem_desc_sw128_split(sb + C::S_RING, 16, 1024);
-            const uint32_t blk_bytes = (uint32_t)R * 128u;
-            int ki = 0;
+            // K slots are group-major: 8-row groups 9 KB apart, column blocks 1 KB apart.  A
+            // chunk is one N = 64 operand at any page size, and an even chunk whose successor
+            // sits in the next slot forms with it one N = 128 operand (16 groups 9 KB apart)
+            // whose scores fill both S buffers: half the MMAs for two of every three pairs.
+            const uint32_t IDESC64 = idesc_bf16_f32(128, 64, false);
+            const uint32_t IDESC128 = idesc_bf16_f32(128, 128, false);
+            const SmemDesc dK = smem_desc_sw128_split(sb + C::S_RING, 16, 9u * 1024u);
             bool ok = n_chunks > 0 && mbar_wait(sBar + C::B_QREADY, 0, abort_flag);
             tc_fence_after();
-            for (int j = 0; ok && j < n_chunks; ++j) {
-                const int ps = j & 1;
-                if (!mbar_wait(sBar + C::B_SFREE + 8 * ps, ((j >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                for (int t = 0; t < C::KLOADS; ++t) {
-                    const int st = ki % C::RK;
-                    if (!mbar_wait(sBar + C::B_KFULL + 8 * st, (ki / C::RK) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const SmemDesc bk{dK.lo + ((st * C::KSLOT) >> 4), dK.hi};
-                    for (int pp = 0; pp < np; ++pp) {
-                        const uint32_t d = tmem + 64u * (uint32_t)ps + (uint32_t)(pp * R);
-                        for (int cc = 0; cc < C::KB; ++cc) {
-                            const int c = C::KB * t + cc;
-                            const uint32_t boff = (uint32_t)(pp * C::KB + cc) * blk_bytes;
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                tc_mma_ts(d, tmem + C::T_Q + 32u * c + 8u * kk, desc_at(bk, boff + kk * 32u), IDESC,
-                                          (c | kk) ? 1u : 0u);
-                        }
-                    }
-                    tc_commit(sBar + C::B_KEMPTY + 8 * st);
-                    ++ki;
+            for (int j = 0; ok && j < n_chunks;) {
+                const int st = j % C::RK;  // one K load per chunk: load index = chunk index
+                const bool pair = (j & 1) == 0 && j + 1 < n_chunks && st + 1 < C::RK;
+                const int nc = pair ? 2 : 1;
+                for (int q = 0; ok && q < nc; ++q) {
+                    const int jj = j + q;
+                    ok = mbar_wait(sBar + C::B_SFREE + 8 * (jj & 1), ((jj >> 1) & 1) ^ 1, abort_flag) &&
+                         mbar_wait(sBar + C::B_KFULL + 8 * (jj % C::RK), (jj / C::RK) & 1, abort_flag);
                 }
                 if (!ok) break;
-                tc_commit(sBar + C::B_SFULL + 8 * ps);
+                tc_fence_after();
+                const uint32_t d = tmem + 64u * (uint32_t)(j & 1);
+                const uint32_t base = (uint32_t)st * C::KSLOT;
+                for (int c = 0; c < 9; ++c) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_ts(d, tmem + C::T_Q + 32u * c + 8u * kk, desc_at(dK, base + (uint32_t)c * 1024u + kk * 32u),
+                                  pair ? IDESC128 : IDESC64, (c | kk) ? 1u : 0u);
+                }
+                for (int q = 0; q < nc; ++q) {
+                    tc_commit(sBar + C::B_KEMPTY + 8 * ((j + q) % C::RK));
+                    tc_commit(sBar + C::B_SFULL + 8 * ((j + q) & 1));
+                }
+                j += nc;
             }
             tc_commit(sBar + C::B_SDRAIN);
             mbar_wait(sBar + C::B_SDRAIN, 0, nullptr, 100000000ull);
