@@ -215,8 +215,10 @@ size_t attn_fwd_ragged_noalloc_max_scratch(void);
  *   Absorbed MLA: pass v_pool == k_pool with Dv < Dqk; V is then the first Dv
  *   columns of each K row ("cuDNN Frontend v1.32.0 Release Notes", "SDPA:
  *   wider native forward support": Q/K576, V512, absorbed-MLA cache layouts).
- *   MLA (Dqk 576, Dv 512) needs Hkv == 1 and page_size 16, 32 or a multiple
- *   of 64 (ATTN_ERR_UNSUPPORTED otherwise); any Hq (groups of 128 heads).
+ *   MLA (Dqk 576, Dv 512) needs Hkv == 1, page_size 16, 32 or a multiple of
+ *   64, and a K pool whose page stride is a whole number of 8-row groups
+ *   (k_pool_strides[0] % (8 * k_pool_strides[1]) == 0; dense pools qualify)
+ *   (ATTN_ERR_UNSUPPORTED otherwise); any Hq (groups of 128 heads).
  *   GQA needs page_size dividing or divisible by 64 (at least 8) and
  *   Hq / Hkv <= 16.
  *   Each page-table row holds at least ceil(max_kv_len / page_size) entries.
