@@ -91,28 +91,6 @@ int setup_device(int* dev_out, int* sms_out) {
     return ATTN_OK;
 }
 
-// 4D bf16 tensor map with 128-byte swizzle.  dims/strides: innermost first;
-// strides in ELEMENTS for dims 1..3.  Box inner extent is 64 elements (128 B).
-int encode_4d(CUtensorMap* map, const void* base, const uint64_t dims[4], const int64_t strides_el[3],
-              const uint32_t box[4]) {
-    cuuint64_t gdim[4], gstr[3];
-    cuuint32_t bdim[4], estr[4] = {1, 1, 1, 1};
-    for (int i = 0; i < 4; ++i) {
-        if (dims[i] == 0 || dims[i] > (1ull << 32)) return ATTN_ERR_INVALID_ARG;
-        gdim[i] = dims[i];
-        bdim[i] = box[i];
-    }
-    for (int i = 0; i < 3; ++i) {
-        const int64_t bytes = strides_el[i] * 2;
-        if (bytes <= 0 || (bytes % 16) != 0 || bytes >= (int64_t(1) << 40)) return ATTN_ERR_INVALID_ARG;
-        gstr[i] = (cuuint64_t)bytes;
-    }
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), gdim, gstr, bdim,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_INVALID_ARG;
-}
-
 // 5D bf16 tensor map with 128-byte swizzle; strides in BYTES for dims 1..4.
 int encode_5d(CUtensorMap* map, const void* base, const uint64_t dims[5], const int64_t strides_b[4],
               const uint32_t box[5]) {
