@@ -242,42 +242,25 @@ int launch_decode_schedule(DecodeParams& dp, char* wsb, const SplitWs& w, int64_
 }
 
 // Launches the GQA decode kernel with RT 16-row m-tiles (1, 2 or 4): grid
-// (1, Hkv, B) without splits, one block per scheduled piece with them (then
-// with programmatic stream serialization after the schedule kernel).  A
+// (1, Hkv, B) without splits, one block per scheduled piece with them.  A
 // launch of at most one block per SM gets the 6-stage ring (RT 1).
-template <typename Kernel>
-int launch_decode_ex(Kernel kernel, dim3 grid, uint32_t smem, bool early, const DecodeParams& dp, cudaStream_t st) {
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(160, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = early ? attr : nullptr;
-    cfg.numAttrs = early ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, dp) == cudaSuccess ? launch_status() : ATTN_ERR_LAUNCH;
-}
-
 int launch_decode_gqa(const DecodeParams& dp, int D, int RT, dim3 grid, int sms, cudaStream_t st) {
-    // after the split schedule, the decode's blocks may start while it runs (they wait for
-    // its records on the device)
-    const bool early = dp.segs != nullptr;
     const int64_t blocks = (int64_t)grid.x * grid.y * grid.z;
     if (RT == 1 && blocks <= sms) {
-        if (D == 128) return launch_decode_ex(b2::decode_gqa_kernel<128, 1, 6>, grid, b2::DecodeCfg<128, 6>::SMEM, early, dp, st);
-        return launch_decode_ex(b2::decode_gqa_kernel<64, 1, 6>, grid, b2::DecodeCfg<64, 6>::SMEM, early, dp, st);
+        if (D == 128) b2::decode_gqa_kernel<128, 1, 6><<<grid, 160, b2::DecodeCfg<128, 6>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<64, 1, 6><<<grid, 160, b2::DecodeCfg<64, 6>::SMEM, st>>>(dp);
+        return launch_status();
     }
     if (D == 128) {
-        if (RT == 1) return launch_decode_ex(b2::decode_gqa_kernel<128, 1>, grid, b2::DecodeCfg<128>::SMEM, early, dp, st);
-        if (RT == 2) return launch_decode_ex(b2::decode_gqa_kernel<128, 2>, grid, b2::DecodeCfg<128>::SMEM, early, dp, st);
-        return launch_decode_ex(b2::decode_gqa_kernel<128, 4>, grid, b2::DecodeCfg<128>::SMEM, early, dp, st);
+        if (RT == 1) b2::decode_gqa_kernel<128, 1><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+        else if (RT == 2) b2::decode_gqa_kernel<128, 2><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<128, 4><<<grid, 160, b2::DecodeCfg<128>::SMEM, st>>>(dp);
+    } else {
+        if (RT == 1) b2::decode_gqa_kernel<64, 1><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+        else if (RT == 2) b2::decode_gqa_kernel<64, 2><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
+        else b2::decode_gqa_kernel<64, 4><<<grid, 160, b2::DecodeCfg<64>::SMEM, st>>>(dp);
     }
-    if (RT == 1) return launch_decode_ex(b2::decode_gqa_kernel<64, 1>, grid, b2::DecodeCfg<64>::SMEM, early, dp, st);
-    if (RT == 2) return launch_decode_ex(b2::decode_gqa_kernel<64, 2>, grid, b2::DecodeCfg<64>::SMEM, early, dp, st);
-    return launch_decode_ex(b2::decode_gqa_kernel<64, 4>, grid, b2::DecodeCfg<64>::SMEM, early, dp, st);
+    return launch_status();
 }
 
 // GQA decode maps over a pool: (column in block, slot, 64-column block, head,

@@ -201,9 +201,6 @@ __global__ void __launch_bounds__(1024) decode_schedule_kernel(const __grid_cons
                                                                DecodeSeg* __restrict__ segs, int* __restrict__ ctr) {
     __shared__ int hist[kSortBuckets];
     __shared__ int warp_sums[32];
-    // the decode launch that follows may start its blocks now: they wait for this kernel
-    // (griddep_wait) before reading its output
-    griddep_launch_dependents();
     const int tid = threadIdx.x;
     const int Hkv = p.Hkv, S = p.num_splits;
     auto bucket = [&](int n) { return kSortBuckets - 1 - min(kSortBuckets - 1, n >> shift); };
@@ -408,7 +405,6 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
     // blockIdx.y of sequence blockIdx.z, all of its keys
     DecodeSeg sg;
     if (p.segs != nullptr) {
-        griddep_wait();  // the schedule kernel's records (launched right after it, possibly early)
         const int4* r = reinterpret_cast<const int4*>(p.segs + blockIdx.x);
         const int4 a = __ldg(r);
         if (a.x < 0) return;  // no piece for this block, before any barrier exists

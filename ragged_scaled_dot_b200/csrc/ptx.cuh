@@ -161,14 +161,6 @@ __device__ __forceinline__ void st_async_peer_b32(uint32_t dst_cluster, uint32_t
                  : "memory");
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start while the kernel before it runs; griddep_wait blocks
-// until that kernel has completed and its memory is visible (a no-op for a
-// launch without the attribute), and griddep_launch_dependents lets the next
-// kernel's blocks be scheduled early.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // Named-barrier reductions over `count` threads (a multiple of 32, every
 // thread of each participating warp): all wait, all get the AND / OR.
 __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool v) {
