@@ -183,6 +183,8 @@ MIXED = [
     ([1] * 8 + [4] * 8, [100 * i + 1 for i in range(16)], 8, 2, 128, 64, 3, True, rsd.ATTN_LSE_PACKED_TH),
     # short rows over an empty cache and a 1-key cache (the first query of the 2 sees no key)
     ([1, 2, 300, 4], [0, 1, 500, 70], 8, 2, 128, 64, 2, True, rsd.ATTN_LSE_PADDED_BSH),
+    # 64-row (4-query, G 16) pieces of a 60000-key cache merged over two levels of groups of 8
+    ([4, 2, 700], [60000, 30000, 2000], 32, 2, 64, 16, 64, True, rsd.ATTN_LSE_PACKED_TH),
 ]
 
 
