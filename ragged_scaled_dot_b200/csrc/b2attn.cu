@@ -672,7 +672,7 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
     std::memset(&dp, 0, sizeof(dp));
     // short rows: G * qmax query rows in RT m16 tiles; with splits, one block per piece
     int RT = 1;
-    int64_t n_cta = 0;
+    int64_t n_split_blocks = 0;
     const int64_t dec_pairs = (int64_t)B * Hkv;
     if (qmax > 0) {
         if (int e = encode_decode_pool_maps(dp, k_pool, v_pool, D, D, page_size, Hkv, num_pages, k_pool_strides,
@@ -681,8 +681,8 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         RT = (G * qmax + 15) / 16;
         if (RT == 3) RT = 4;
         if (num_splits > 1) {
-            n_cta = split_blocks(dec_pairs, max_kv_len, num_splits);
-            if (n_cta == 0) return ATTN_ERR_UNSUPPORTED;
+            n_split_blocks = split_blocks(dec_pairs, max_kv_len, num_splits);
+            if (n_split_blocks == 0) return ATTN_ERR_UNSUPPORTED;
         }
     }
 
@@ -718,8 +718,8 @@ int attn_fwd_paged_prefill_kv_tables(const void* q, const void* k_pool, const vo
         dp.lse_hs = total_q;
         dp.lse_log2 = (lse_layout & ATTN_LSE_LOG2) ? 1 : 0;
         if (num_splits > 1) {
-            if (int e = launch_decode_schedule(dp, wsb, wl.sw, n_cta, max_kv_len, st)) return e;
-            if (int e = launch_decode_gqa(dp, D, RT, dim3((unsigned)n_cta, 1, 1), sms, st)) return e;
+            if (int e = launch_decode_schedule(dp, wsb, wl.sw, n_split_blocks, max_kv_len, st)) return e;
+            if (int e = launch_decode_gqa(dp, D, RT, dim3((unsigned)n_split_blocks, 1, 1), sms, st)) return e;
         } else {
             if (int e = launch_decode_gqa(dp, D, RT, dim3(1, Hkv, B), sms, st)) return e;
         }
@@ -901,10 +901,10 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     const int64_t mla_units = (int64_t)B * num_splits * ((Hq + 127) / 128);
     if (mla && 2 * mla_units > 0x7fffffff) return ATTN_ERR_UNSUPPORTED;
     // GQA with splits: one block per scheduled piece
-    int64_t n_cta = 0;
+    int64_t n_split_blocks = 0;
     if (!mla && num_splits > 1) {
-        n_cta = split_blocks((int64_t)B * Hkv, max_kv_len, num_splits);
-        if (n_cta == 0) return ATTN_ERR_UNSUPPORTED;
+        n_split_blocks = split_blocks((int64_t)B * Hkv, max_kv_len, num_splits);
+        if (n_split_blocks == 0) return ATTN_ERR_UNSUPPORTED;
     }
 
     DecodeParams dp;
@@ -994,8 +994,8 @@ int attn_fwd_paged_kv_tables(const void* q, const void* k_pool, const void* v_po
     // GQA: the G <= 16 query heads of a KV head fill one m16 tile
     if (num_splits > 1) {
         const SplitWs sw = split_ws_layout(0, B, R, 1, Dv, num_splits);
-        if (int e = launch_decode_schedule(dp, wsb, sw, n_cta, max_kv_len, st)) return e;
-        return launch_decode_gqa(dp, Dqk, 1, dim3((unsigned)n_cta, 1, 1), sms, st);
+        if (int e = launch_decode_schedule(dp, wsb, sw, n_split_blocks, max_kv_len, st)) return e;
+        return launch_decode_gqa(dp, Dqk, 1, dim3((unsigned)n_split_blocks, 1, 1), sms, st);
     }
     return launch_decode_gqa(dp, Dqk, 1, dim3(1, Hkv, B), sms, st);
 }
