@@ -132,10 +132,10 @@ __device__ __forceinline__ uint32_t decode_chunk_bytes(const DecodeParams& p, in
 // all column blocks of those rows, landing at dst + i * (ncol_blocks * box_rows *
 // 128) as [column block][rows][128 B] (for box_rows 64: the [column block][64
 // rows] tile).  All page ids of the chunk are read before any box is issued, so
-// their latencies overlap (each TMA issue is ordered after the reads before it;
-// one thread reading them box by box could not keep a small batch's few blocks
-// streaming), and with one page table for K and V the V boxes reuse the K
-// boxes' ids.
+// their latencies overlap (each TMA issue is ordered after the reads before it),
+// and with one page table for K and V the V boxes reuse the K boxes' ids.  One
+// thread issues them; the kernel uses this for pages of 64 keys or more (NB = 1),
+// and decode_produce_small_pages below for smaller pages.
 template <int NB>
 __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t dst_k, uint32_t dst_v, uint32_t bar,
                                                 int b, int g, int t0, int hi, int ncol_blocks,
@@ -172,6 +172,53 @@ __device__ __forceinline__ void decode_issue_kv(const DecodeParams& p, uint32_t 
             tma_load_5d(dst_v + i * box_bytes, &p.tm_v, bar, 0, slot, 0, g, pv);
         }
     }
+}
+
+// Pages of fewer than 64 keys: the producer warp issues a chunk's boxes together,
+// lane i < NB K box i and lane NB + i V box i (NB = 64 / box_rows), each lane reading
+// its own page id (from the piece's window, else the table; V boxes read the K ids
+// when K and V share a table).  One thread issuing the 8 boxes of a page-16 chunk
+// one after another spent ~275 cycles a box, longer than the compute warps take to
+// consume the chunk.  Kept out of line so the whole-page loop stays as it was (the
+// warp-wide loop made that one slower).  Returns the chunks issued.
+template <int NST>
+__device__ __noinline__ int decode_produce_small_pages(const DecodeParams& p, uint32_t sBar, volatile int* abort_flag,
+                                                       uint32_t sb, uint32_t stage_bytes, uint32_t chunk_bytes,
+                                                       int ncb, int b, int g, int lo, int hi, int n_chunks,
+                                                       const volatile int* ids_k, const volatile int* ids_v, int p0,
+                                                       int nids, int lane) {
+    const int R = p.box_rows;
+    const int NB = 64 / R;
+    const bool is_v = lane >= NB;
+    const int i = is_v ? lane - NB : lane;
+    const bool v_table = is_v && !(p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride);
+    const uint32_t box_bytes = (uint32_t)(ncb * R) * 128u;
+    int cc = 0;
+    for (; cc < n_chunks; ++cc) {
+        const int st = cc % NST;
+        const uint32_t full = sBar + 8u * st, empty = sBar + 8u * (NST + st);
+        const int t0 = lo + cc * 64;  // t0 >= hi only for the keyless unit of an empty sequence
+        bool w_ok = true;
+        if (lane == 0) {
+            w_ok = mbar_wait(empty, ((cc / NST) & 1) ^ 1, abort_flag);
+            if (w_ok) mbar_arrive_expect_tx(full, t0 < hi ? decode_chunk_bytes(p, t0, hi, ncb, 2) : 0u);
+        }
+        // the stage is free and its byte count set before any lane issues a box
+        if (!__shfl_sync(0xffffffffu, w_ok ? 1 : 0, 0)) break;
+        const int t = t0 + i * R;
+        if (lane < 2 * NB && t < hi) {
+            const int w = t / p.page_size - p0;  // position in the window of shared-memory ids
+            int id;
+            if (w < nids) id = v_table ? ids_v[w] : ids_k[w];
+            else if (v_table) id = page_lookup(p.v_page_table, p.v_pt_stride, b, t, p.page_size);
+            else id = page_lookup(p.page_table, p.pt_stride, b, t, p.page_size);
+            // out of range: page -1, and TMA fills the box with zeros
+            const int page = page_checked(id, p.num_pages);
+            const uint32_t dst = sb + st * stage_bytes + (is_v ? chunk_bytes : 0u) + i * box_bytes;
+            tma_load_5d(dst, is_v ? &p.tm_v : &p.tm_k, full, 0, page_slot(t, p.page_size), 0, g, page);
+        }
+    }
+    return cc;
 }
 
 // Byte offset of key row k of a chunk's K (or V) tile, column block 0: page box
@@ -479,31 +526,17 @@ __global__ void __launch_bounds__(160, NST_ <= 3 ? 2 : 1) decode_gqa_kernel(cons
         }
         __syncwarp();
         int cc = 0;  // chunks issued
-        if (lane == 0) {
+        if (p.box_rows < 64) {
+            cc = decode_produce_small_pages<NST>(p, sBar, abort_flag, sb, C::STAGE, C::CHUNK, C::NCB, b, g, lo, hi,
+                                                 n_chunks, ids_k, ids_v, p0, nids, lane);
+        } else if (lane == 0) {
             for (; cc < n_chunks; ++cc) {
                 const int st = cc % NST;
                 if (!mbar_wait(empty_bar(st), ((cc / NST) & 1) ^ 1, abort_flag)) break;
                 const int t0 = lo + cc * 64;  // t0 >= hi only for the keyless unit of an empty sequence
                 mbar_arrive_expect_tx(full_bar(st), t0 < hi ? decode_chunk_bytes(p, t0, hi, C::NCB, 2) : 0u);
                 const uint32_t dst = sb + st * C::STAGE;
-                switch (64 / p.box_rows) {
-                    case 1:
-                        decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
-                                           p0, nids);
-                        break;
-                    case 2:
-                        decode_issue_kv<2>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
-                                           p0, nids);
-                        break;
-                    case 4:
-                        decode_issue_kv<4>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
-                                           p0, nids);
-                        break;
-                    default:
-                        decode_issue_kv<8>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v,
-                                           p0, nids);
-                        break;
-                }
+                decode_issue_kv<1>(p, dst, dst + C::CHUNK, full_bar(st), b, g, t0, hi, C::NCB, ids_k, ids_v, p0, nids);
             }
         }
         // drain: every issued load lands before the block leaves
