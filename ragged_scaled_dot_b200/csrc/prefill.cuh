@@ -193,6 +193,106 @@ __device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int 
     return t0 < Lkv && Lkv <= t0 + 128 && (Lkv % p.box_rows) != 0;
 }
 
+// Mode 2 with pages of fewer than 64 keys: the whole producer warp runs the
+// scheduler and load loop.  Lane 0 claims items, publishes them, loads Q and
+// handles the stage barriers; after a warp shuffle, lane i < 128 / box_rows issues
+// page box i of each K and V tile, reading its own page id, so a tile's 8 (page
+// 16) or 4 (page 32) id reads and box issues overlap.  One thread issuing them one
+// by one, each TMA issue ordered after its id read, could not keep the MMAs fed:
+// pages of 16 and 32 keys ran at 313 and 524 TFLOP/s against 1025 at 64.  Kept
+// out of line, so the page-64 loop keeps its code.  kv_it and q_it return the
+// K/V and Q loads issued (every lane holds the same counts).
+template <int D, int NST, int NRING>
+__device__ __noinline__ void prefill_produce_small_pages(const PrefillParams& p, uint32_t sQ, uint32_t sKV,
+                                                         uint32_t sBar, uint32_t b_qfull, uint32_t b_qempty,
+                                                         uint32_t b_ifull0, uint32_t b_iempty0, uint32_t b_vtail0,
+                                                         volatile int* item_ring, volatile int* abort_flag,
+                                                         uint8_t* kv_gen, int lane, int& kv_it, int& q_it) {
+    constexpr uint32_t TILE = (D / 64) * 16384u;
+    constexpr unsigned FULL = 0xffffffffu;
+    const int R = p.box_rows;
+    const int nb = 128 / R;  // page boxes per K or V tile
+    const uint32_t box_bytes = (uint32_t)R * (D / 64) * 128u;
+    const int n_items = p.header[0];
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+        const int r = k % NRING;
+        int idx = -1;
+        bool w_ok = true;
+        if (lane == 0) {
+            w_ok = mbar_wait(b_iempty0 + 8 * r, ((k / NRING) & 1) ^ 1, abort_flag);
+            if (w_ok) {
+                idx = atomicAdd(p.header + 1, 1);
+                if (idx >= n_items) idx = -1;
+                item_ring[r] = idx;
+                mbar_arrive(b_ifull0 + 8 * r);
+            }
+        }
+        w_ok = __shfl_sync(FULL, w_ok ? 1 : 0, 0) != 0;
+        idx = __shfl_sync(FULL, idx, 0);
+        if (!w_ok || idx < 0) break;
+        PrefillItem it;
+        prefill_get_item(p, idx, it);
+        if (it.n_kv == 0) continue;
+        if (lane == 0) {
+            w_ok = mbar_wait(b_qempty, (q_it & 1) ^ 1, abort_flag);
+            if (w_ok) {
+                mbar_arrive_expect_tx(b_qfull, it.nh * TILE);
+                for (int s = 0; s < it.nh; ++s)
+                    tma_load_5d(sQ + s * TILE, &p.tm_q, b_qfull, 0, it.q_tok0, 0, it.h0 + s, it.batch);
+            }
+        }
+        if (!__shfl_sync(FULL, w_ok ? 1 : 0, 0)) break;
+        ++q_it;
+        const int g = it.h0 / p.G;
+        for (int j = 0; ok && j < it.n_kv; ++j) {
+            for (int t = 0; t < 2; ++t) {
+                const int st = kv_it % NST;
+                const uint32_t full = sBar + 8u * st, empty = sBar + 8u * (NST + st);
+                if (lane == 0) {
+                    w_ok = mbar_wait(empty, ((kv_it / NST) & 1) ^ 1, abort_flag);
+                    if (w_ok) mbar_arrive_expect_tx(full, TILE);
+                }
+                // the stage is free and its byte count set before any lane issues a box
+                if (!__shfl_sync(FULL, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                if (lane < nb) {
+                    // boxes at or past Lkv (or with a bad page id, recorded) read zeros
+                    const int tk = j * 128 + lane * R;
+                    int gg = p.n_groups;
+                    if (tk < it.Lkv) {
+                        const int32_t* table = t ? p.v_page_table : p.page_table;
+                        const int64_t stride = t ? p.v_pt_stride : p.pt_stride;
+                        const int page = page_checked(page_lookup(table, stride, it.b, tk, p.page_size), p.num_pages);
+                        if (page >= 0) gg = page_group(page, page_slot(tk, p.page_size), p.groups_per_page);
+                    }
+                    tma_load_5d(sKV + st * TILE + (uint32_t)lane * box_bytes, t ? &p.tm_v : &p.tm_k, full, 0, 0, 0,
+                                gg, g);
+                }
+                if (t == 1 && paged_tile_has_tail(p, j * 128, it.Lkv)) {
+                    // value rows past the sequence: zeroed once the tile lands, then the
+                    // tile goes to the MMA thread through this stage's tail barrier
+                    if (lane == 0) {
+                        w_ok = mbar_wait(full, (kv_it / NST) & 1, abort_flag);
+                        if (w_ok) {
+                            uint8_t* vt = kv_gen + st * TILE;
+                            const int r0 = it.Lkv - j * 128;  // rows of the partially valid box past Lkv
+                            const int r1 = min(128, (r0 + R - 1) / R * R);
+                            for (int rr = r0; rr < r1; ++rr)
+                                for (int c = 0; c < (D / 64) * 8; ++c)
+                                    *reinterpret_cast<uint4*>(vt + (rr >> 3) * (D / 64) * 1024 + (c >> 3) * 1024 +
+                                                              (rr & 7) * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
+                            fence_proxy_async_smem();
+                            mbar_arrive(b_vtail0 + 8 * st);
+                        }
+                    }
+                    if (!__shfl_sync(FULL, w_ok ? 1 : 0, 0)) { ok = false; break; }
+                }
+                ++kv_it;
+            }
+        }
+    }
+}
+
 template <int D>
 struct PrefillCfg {
     static constexpr int HALVES = D / 64;
@@ -286,7 +386,19 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
         return idx;
     };
 
-    if (warp == 0 && lane == 0) {
+    if (PAGED && warp == 0 && p.box_rows < 64) {
+        // ------------------------------- scheduler + producer, pages under 64 keys
+        int kv_it = 0, q_it = 0;
+        prefill_produce_small_pages<D, NST, NRING>(p, sQ, sKV, sBar, b_qfull, b_qempty, b_ifull0, b_iempty0, b_vtail0,
+                                                   item_ring, abort_flag, sgen + (sKV - sb), lane, kv_it, q_it);
+        // Let every load the warp issued land before the block exits.
+        if (lane == 0) {
+            const int n_last = min(kv_it, NST);
+            for (int kk = kv_it - n_last; kk < kv_it; ++kk)
+                mbar_wait(full_bar(kk % NST), (kk / NST) & 1, nullptr, 100000000ull);
+            if (q_it > 0) mbar_wait(b_qfull, (q_it - 1) & 1, nullptr, 100000000ull);
+        }
+    } else if (warp == 0 && lane == 0) {
         // ---------------------------------------------- scheduler + producer
         const int n_items = p.header[0];
         int kv_it = 0, q_it = 0;
