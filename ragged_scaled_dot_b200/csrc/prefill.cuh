@@ -14,12 +14,10 @@
 // Warp roles (320 threads):
 //   warp 0      claims items, publishes them to the other roles through a
 //               small shared-memory ring, and issues the TMA loads: Q tiles of
-//               the item, then K(j), V(j) into a ring of NST stages.  Over a
-//               paged cache it also reads the page ids; with 64-row page boxes
-//               a tile's two ids are read together, the V boxes reuse the K
-//               boxes' ids, and the next tile's ids are read while it waits for
-//               a free stage (one thread doing these reads one by one could not
-//               keep up with the MMAs).
+//               the item, then K(j), V(j) into a ring of NST stages (one thread).
+//               Over a paged cache the whole warp runs this loop: each lane
+//               reads one page id of a tile and issues its page box, so the
+//               id reads and box issues of a tile overlap.
 //   warp 1      owns TMEM; one thread issues every tcgen05.mma and commit
 //               (descriptor bases are precomputed: this thread shares its SM
 //               sub-partition with two busy softmax warps, so every instruction
@@ -146,46 +144,9 @@ __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx
 
 // Mode 2 K/V tile of 128 keys from t0: 128 / box_rows page boxes, each
 // (64 columns, 8 rows, D/64 blocks, box_rows/8 groups, 1 head) landing as
-// [group][block][8 rows][128 B].  Two 64-row boxes placed back to back keep
-// one uniform 8-row-group stride, so the tile is a single MMA operand across
-// pages.  Boxes at or past Lkv (or with a bad page id, recorded) read zeros.
-__device__ __forceinline__ void paged_issue_tile(const PrefillParams& p, const CUtensorMap* map,
-                                                 const int32_t* table, int64_t table_stride, uint32_t dst,
-                                                 uint32_t bar, int b, int g, int t0, int Lkv, uint32_t box_bytes) {
-    for (int i = 0; i < 128 / p.box_rows; ++i) {
-        const int t = t0 + i * p.box_rows;
-        int gg = p.n_groups;
-        if (t < Lkv) {
-            const int page = page_checked(page_lookup(table, table_stride, b, t, p.page_size), p.num_pages);
-            if (page >= 0) gg = page_group(page, page_slot(t, p.page_size), p.groups_per_page);
-        }
-        tma_load_5d(dst + (uint32_t)i * box_bytes, map, bar, 0, 0, 0, gg, g);
-    }
-}
-
-// Mode 2 with two page boxes per tile (64-row boxes, the common page size): both
-// page ids are read before either box is issued, so their latencies overlap
-// (each TMA issue is ordered after the reads before it).  id = -1 past Lkv.
-__device__ __forceinline__ void paged_tile_ids2(const PrefillParams& p, const int32_t* table, int64_t table_stride,
-                                                int b, int t0, int Lkv, int (&id)[2]) {
-    const int t1 = t0 + p.box_rows;
-    id[0] = (t0 < Lkv) ? page_lookup(table, table_stride, b, t0, p.page_size) : -1;
-    id[1] = (t1 < Lkv) ? page_lookup(table, table_stride, b, t1, p.page_size) : -1;
-}
-__device__ __forceinline__ void paged_issue_ids2(const PrefillParams& p, const CUtensorMap* map, const int (&id)[2],
-                                                 uint32_t dst, uint32_t bar, int g, int t0, int Lkv,
-                                                 uint32_t box_bytes) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int t = t0 + i * p.box_rows;
-        int gg = p.n_groups;
-        if (t < Lkv) {
-            const int page = page_checked(id[i], p.num_pages);
-            if (page >= 0) gg = page_group(page, page_slot(t, p.page_size), p.groups_per_page);
-        }
-        tma_load_5d(dst + (uint32_t)i * box_bytes, map, bar, 0, 0, 0, gg, g);
-    }
-}
+// [group][block][8 rows][128 B].  Boxes placed back to back keep one uniform
+// 8-row-group stride, so the tile is a single MMA operand across pages.  Boxes at
+// or past Lkv (or with a bad page id, recorded) read zeros.
 
 // Mode 2: does the K/V tile from t0 end inside a page box that runs past Lkv
 // (rows past the sequence that can hold stale values, possibly NaN)?
@@ -193,17 +154,18 @@ __device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int 
     return t0 < Lkv && Lkv <= t0 + 128 && (Lkv % p.box_rows) != 0;
 }
 
-// Mode 2 with pages of fewer than 64 keys: the whole producer warp runs the
-// scheduler and load loop.  Lane 0 claims items, publishes them, loads Q and
-// handles the stage barriers; after a warp shuffle, lane i < 128 / box_rows issues
-// page box i of each K and V tile, reading its own page id, so a tile's 8 (page
-// 16) or 4 (page 32) id reads and box issues overlap.  One thread issuing them one
-// by one, each TMA issue ordered after its id read, could not keep the MMAs fed:
-// pages of 16 and 32 keys ran at 313 and 524 TFLOP/s against 1025 at 64.  Kept
-// out of line, so the page-64 loop keeps its code.  kv_it and q_it return the
-// K/V and Q loads issued (every lane holds the same counts).
+// Mode 2 scheduler and producer, run by the whole producer warp.  Lane 0 claims
+// items, publishes them, loads Q and handles the stage barriers; after a warp
+// shuffle, lane i < 128 / box_rows issues page box i of each K and V tile, reading
+// its own page id, so a tile's id reads and box issues overlap.  One thread issuing
+// the boxes one by one, each TMA issue ordered after its id read, could not keep
+// the MMAs fed: with it, 4 chunks of 1024 queries ran at 313, 525, 1030 and 1031
+// TFLOP/s with pages of 16, 32, 64 and 128 keys, and with the warp at 963, 1071,
+// 1071 and 1040.  Kept out of line (the kernel's other roles keep their code).
+// kv_it and q_it return the K/V and Q loads issued (every lane holds the same
+// counts).
 template <int D, int NST, int NRING>
-__device__ __noinline__ void prefill_produce_small_pages(const PrefillParams& p, uint32_t sQ, uint32_t sKV,
+__device__ __noinline__ void prefill_produce_paged(const PrefillParams& p, uint32_t sQ, uint32_t sKV,
                                                          uint32_t sBar, uint32_t b_qfull, uint32_t b_qempty,
                                                          uint32_t b_ifull0, uint32_t b_iempty0, uint32_t b_vtail0,
                                                          volatile int* item_ring, volatile int* abort_flag,
@@ -386,11 +348,11 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
         return idx;
     };
 
-    if (PAGED && warp == 0 && p.box_rows < 64) {
-        // ------------------------------- scheduler + producer, pages under 64 keys
+    if (PAGED && warp == 0) {
+        // ------------------------------------ scheduler + producer over a paged cache
         int kv_it = 0, q_it = 0;
-        prefill_produce_small_pages<D, NST, NRING>(p, sQ, sKV, sBar, b_qfull, b_qempty, b_ifull0, b_iempty0, b_vtail0,
-                                                   item_ring, abort_flag, sgen + (sKV - sb), lane, kv_it, q_it);
+        prefill_produce_paged<D, NST, NRING>(p, sQ, sKV, sBar, b_qfull, b_qempty, b_ifull0, b_iempty0, b_vtail0,
+                                             item_ring, abort_flag, sgen + (sKV - sb), lane, kv_it, q_it);
         // Let every load the warp issued land before the block exits.
         if (lane == 0) {
             const int n_last = min(kv_it, NST);
@@ -399,7 +361,7 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
             if (q_it > 0) mbar_wait(b_qfull, (q_it - 1) & 1, nullptr, 100000000ull);
         }
     } else if (warp == 0 && lane == 0) {
-        // ---------------------------------------------- scheduler + producer
+        // ------------------------------------------- scheduler + producer (dense, ragged)
         const int n_items = p.header[0];
         int kv_it = 0, q_it = 0;
         bool ok = true;
@@ -420,56 +382,13 @@ __global__ void __launch_bounds__(320, 1) prefill_kernel(const __grid_constant__
                 tma_load_5d(sQ + s * TILE, &p.tm_q, b_qfull, 0, it.q_tok0, 0, it.h0 + s, it.batch);
             ++q_it;
             const int g = it.h0 / p.G;
-            // with one table for K and V, the V boxes of a tile reuse the K boxes' page ids
-            const bool shared_table = p.v_page_table == p.page_table && p.v_pt_stride == p.pt_stride;
-            // page ids of the next tile, read while this thread waits for a free stage
-            int ids_next[2] = {-1, -1};
-            bool have_next = false;
             for (int j = 0; ok && j < it.n_kv; ++j) {
-                int ids[2] = {-1, -1};
                 for (int t = 0; t < 2; ++t) {
                     const int st = kv_it % NST;
                     if (!mbar_wait(empty_bar(st), ((kv_it / NST) & 1) ^ 1, abort_flag)) { ok = false; break; }
                     mbar_arrive_expect_tx(full_bar(st), TILE);
-                    const CUtensorMap* map = t ? &p.tm_v : &p.tm_k;
-                    if constexpr (PAGED) {
-                        const uint32_t box_bytes = (uint32_t)p.box_rows * (D / 64) * 128u;
-                        if (p.box_rows == 64) {
-                            if (t == 0 && have_next) {
-                                ids[0] = ids_next[0];
-                                ids[1] = ids_next[1];
-                            } else if (t == 0 || !shared_table) {
-                                paged_tile_ids2(p, t ? p.v_page_table : p.page_table, t ? p.v_pt_stride : p.pt_stride,
-                                                it.b, j * 128, it.Lkv, ids);
-                            }
-                            paged_issue_ids2(p, map, ids, sKV + st * TILE, full_bar(st), g, j * 128, it.Lkv, box_bytes);
-                            if (t == 1) {
-                                have_next = j + 1 < it.n_kv;
-                                if (have_next)
-                                    paged_tile_ids2(p, p.page_table, p.pt_stride, it.b, (j + 1) * 128, it.Lkv, ids_next);
-                            }
-                        } else {
-                            paged_issue_tile(p, map, t ? p.v_page_table : p.page_table,
-                                             t ? p.v_pt_stride : p.pt_stride, sKV + st * TILE, full_bar(st), it.b, g,
-                                             j * 128, it.Lkv, box_bytes);
-                        }
-                        if (t == 1 && paged_tile_has_tail(p, j * 128, it.Lkv)) {
-                            // value rows past the sequence: zero them once the tile lands, then
-                            // release the tile to the MMA thread through this stage's tail barrier
-                            if (!mbar_wait(full_bar(st), (kv_it / NST) & 1, abort_flag)) { ok = false; break; }
-                            uint8_t* vt = sgen + (sKV - sb) + st * TILE;
-                            const int r0 = it.Lkv - j * 128;  // rows of the partially valid box past Lkv
-                            const int r1 = min(128, (r0 + p.box_rows - 1) / p.box_rows * p.box_rows);
-                            for (int r = r0; r < r1; ++r)
-                                for (int c = 0; c < (D / 64) * 8; ++c)
-                                    *reinterpret_cast<uint4*>(vt + (r >> 3) * (D / 64) * 1024 + (c >> 3) * 1024 +
-                                                              (r & 7) * 128 + (c & 7) * 16) = make_uint4(0, 0, 0, 0);
-                            fence_proxy_async_smem();
-                            mbar_arrive(b_vtail0 + 8 * st);
-                        }
-                    } else {
-                        tma_load_5d(sKV + st * TILE, map, full_bar(st), 0, it.kv_tok0 + j * 128, 0, g, it.batch);
-                    }
+                    tma_load_5d(sKV + st * TILE, t ? &p.tm_v : &p.tm_k, full_bar(st), 0, it.kv_tok0 + j * 128, 0, g,
+                                it.batch);
                     ++kv_it;
                 }
             }
