@@ -40,6 +40,8 @@ GQA_CASES = [
     ([100, 1, 777], 32, 4, 64, 32, "HND", 4),
     ([1000, 20], 4, 4, 128, 128, "NHD", 2),
     ([3000], 12, 1, 128, 64, "HND", 16),   # more splits than some sequences have pages
+    ([7, 64, 1000, 333], 16, 2, 128, 8, "HND", 1),   # 8-row pages: 16 lanes issue a chunk's boxes
+    ([300, 45, 2000], 8, 1, 128, 16, "HND", 1),      # page 16 unsplit (the deep ring)
 ]
 
 

@@ -134,13 +134,16 @@ def test_paged_prefill_head_major_base2_lse():
     assert_lse_close(lg, l_ref * LOG2E, "paged prefill, head-major base-2 LSE", atol=LSE_ATOL * LOG2E)
 
 
-def test_paged_prefill_independent_kv_tables():
+@pytest.mark.parametrize("ps", [64, 16])
+def test_paged_prefill_independent_kv_tables(ps):
     """Chunked prefill with V in its own pool and page table: the oracle's
-    result, and bit-identical to one shared table over the original pool."""
-    lens_q, lens_kv, ps = [3, 130, 64], [700, 130, 300], 64
-    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=71)
+    result, and bit-identical to one shared table over the original pool.
+    Page 16 puts 8 page boxes in each K or V tile (one producer lane each, V
+    lanes reading V's table)."""
+    lens_q, lens_kv = [3, 130, 64], [700, 130, 300]
+    q, k, v, table, kl, cu_q = _inputs(lens_q, lens_kv, 8, 2, 128, ps, seed=71 + ps)
     n_pages = [(L + ps - 1) // ps for L in lens_kv]
-    table_v, total = synth.page_table(lens_kv, ps, 73)
+    table_v, total = synth.page_table(lens_kv, ps, 73 + ps)
     v2 = torch.full((total + 4,) + tuple(v.shape[1:]), float("nan"), dtype=v.dtype, device=DEV)
     src = np.concatenate([table[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
     dst = np.concatenate([table_v[b, :n] for b, n in enumerate(n_pages)]).astype(np.int64)
