@@ -1,8 +1,11 @@
 // decode.cuh -- paged-KV decode (one query token per sequence) with split-KV.
 //
-// Pages are gathered with TMA, one box per (page, 64-wide column block): the
-// page table gives the physical page of each logical page ("cuDNN Frontend
-// v1.31.0 Release Notes", "SDPA: paged KV, split-KV, and engine selection").
+// Pages are gathered with TMA, one box per page covering every column block
+// (min(page size, 64) rows): the page table gives the physical page of each
+// logical page ("cuDNN Frontend v1.31.0 Release Notes", "SDPA: paged KV,
+// split-KV, and engine selection").  One producer thread issues a chunk's boxes
+// for pages of 64 keys or more; for smaller pages the producer warp issues them
+// together, one lane per box.
 // Decode is HBM-bound (8 flop per KV byte at Hq/Hkv = 8), so the small
 // contractions run on warp-level MMAs while the memory system streams pages;
 // the G query heads of one KV head are the MMA rows, so every K/V byte is read
