@@ -41,14 +41,14 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # small case, as a ratio to the bytes that scale with the launch, applied to
 # the full launch.  None when the kernel changed after the counters were taken
 # or has no capture.
-#   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.0404 / 1.0611 GB)
+#   ragged_prefill: per Q+K+V+O byte, 16 sequences (1.0432 / 1.0611 GB)
 #   paged_decode: per K/V byte, batch 16, 2 splits (1.3665 / 1.3589 GB)
 #   mla_decode: per K/V byte, batch 8 (0.3439 / 0.3355 GB; the partials grow with the
 #     batch like the K/V bytes)
 #   paged_prefill: per Q+O+K+V byte, 4 chunks of 1024 queries (0.6825 / 0.6345 GB)
-#   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7045 / 0.6711 GB)
-TRAFFIC_RATIO = {"ragged_prefill": 0.9805, "paged_decode": 1.0056, "mla_decode": 1.0262, "paged_prefill": 1.0756,
-                 "dense_prefill": 1.0497}
+#   dense_prefill: per Q+K+V+O byte, the bench's own size, batch 8 (0.7054 / 0.6711 GB)
+TRAFFIC_RATIO = {"ragged_prefill": 0.9831, "paged_decode": 1.0056, "mla_decode": 1.0262, "paged_prefill": 1.0756,
+                 "dense_prefill": 1.0511}
 
 
 def load_peaks():
