@@ -142,12 +142,6 @@ __device__ __forceinline__ void prefill_get_item(const PrefillParams& p, int idx
     it.n_kv = prefill_n_kv(it.qt, it.Lq, it.Lkv, p.causal);
 }
 
-// Mode 2 K/V tile of 128 keys from t0: 128 / box_rows page boxes, each
-// (64 columns, 8 rows, D/64 blocks, box_rows/8 groups, 1 head) landing as
-// [group][block][8 rows][128 B].  Boxes placed back to back keep one uniform
-// 8-row-group stride, so the tile is a single MMA operand across pages.  Boxes at
-// or past Lkv (or with a bad page id, recorded) read zeros.
-
 // Mode 2: does the K/V tile from t0 end inside a page box that runs past Lkv
 // (rows past the sequence that can hold stale values, possibly NaN)?
 __device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int t0, int Lkv) {
@@ -157,19 +151,23 @@ __device__ __forceinline__ bool paged_tile_has_tail(const PrefillParams& p, int 
 // Mode 2 scheduler and producer, run by the whole producer warp.  Lane 0 claims
 // items, publishes them, loads Q and handles the stage barriers; after a warp
 // shuffle, lane i < 128 / box_rows issues page box i of each K and V tile, reading
-// its own page id, so a tile's id reads and box issues overlap.  One thread issuing
+// its own page id, so a tile's id reads and box issues overlap.  A box is (64
+// columns, 8 rows, D/64 blocks, box_rows/8 groups, 1 head) and lands as
+// [group][block][8 rows][128 B]; boxes placed back to back keep one uniform
+// 8-row-group stride, so the tile is a single MMA operand across pages.  Boxes at
+// or past Lkv (or with a bad page id, recorded) read zeros.  One thread issuing
 // the boxes one by one, each TMA issue ordered after its id read, could not keep
-// the MMAs fed: with it, 4 chunks of 1024 queries ran at 313, 525, 1030 and 1031
-// TFLOP/s with pages of 16, 32, 64 and 128 keys, and with the warp at 963, 1071,
-// 1071 and 1040.  Kept out of line (the kernel's other roles keep their code).
+// the MMAs fed: with it, 4 chunks of 1024 queries ran at 313, 525, 1033 and 1035
+// TFLOP/s with pages of 16, 32, 64 and 128 keys, and with the warp at 962, 1089,
+// 1090 and 1094.  Kept out of line (the kernel's other roles keep their code).
 // kv_it and q_it return the K/V and Q loads issued (every lane holds the same
 // counts).
 template <int D, int NST, int NRING>
-__device__ __noinline__ void prefill_produce_paged(const PrefillParams& p, uint32_t sQ, uint32_t sKV,
-                                                         uint32_t sBar, uint32_t b_qfull, uint32_t b_qempty,
-                                                         uint32_t b_ifull0, uint32_t b_iempty0, uint32_t b_vtail0,
-                                                         volatile int* item_ring, volatile int* abort_flag,
-                                                         uint8_t* kv_gen, int lane, int& kv_it, int& q_it) {
+__device__ __noinline__ void prefill_produce_paged(const PrefillParams& p, uint32_t sQ, uint32_t sKV, uint32_t sBar,
+                                                   uint32_t b_qfull, uint32_t b_qempty, uint32_t b_ifull0,
+                                                   uint32_t b_iempty0, uint32_t b_vtail0, volatile int* item_ring,
+                                                   volatile int* abort_flag, uint8_t* kv_gen, int lane, int& kv_it,
+                                                   int& q_it) {
     constexpr uint32_t TILE = (D / 64) * 16384u;
     constexpr unsigned FULL = 0xffffffffu;
     const int R = p.box_rows;
