@@ -25,8 +25,9 @@
 //   warps 2-5   softmax for slot 0 (query head h0), one TMEM lane (row) each:
 //               any four consecutive warps cover the four TMEM lane quadrants.
 //   warps 6-9   softmax for slot 1 (query head h0 + 1).
-// Ten warps (not twelve) leave each thread about 200 registers, enough for a
-// 128-column score row without spilling.
+// Ten warps put three on two of the SM's four sub-partitions, so a thread may
+// hold 168 registers (16384 per sub-partition / 96); the kernel uses 165, enough
+// for a 128-column score row without spilling, and little room for more.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D);
 // P (bf16) overwrites the first 64 columns of its S tile and feeds the PV MMA
 // straight from TMEM.
